@@ -1,0 +1,320 @@
+// Host side of the C ABI declared in include/bcjr.h: argument validation,
+// stream-ordered scratch allocation, kernel selection and launch.
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+
+#include <cuda_runtime.h>
+
+#include "bcjr.h"
+#include "bcjr_kernels.cuh"
+
+namespace {
+
+using bcjr::SweepParams;
+using bcjr::ViterbiParams;
+
+constexpr int kMaxL = 16;
+constexpr int kMaxD = 6;
+constexpr int64_t kMaxLen = 8192;
+constexpr size_t kMaxDynSmem = 227 * 1024;
+
+struct Shape {
+  int L, k, V, D, B, J, S, n;
+  int64_t n_seq, len;
+};
+
+bool fault_alloc() {
+  const char* e = std::getenv("BCJR_FAULT_ALLOC");
+  return e && e[0] == '1';
+}
+
+int check_dev_ptr(const void* p, bool nullable) {
+  if (p == nullptr) return nullable ? BCJR_OK : BCJR_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(p) % 4 != 0) return BCJR_ERR_INVALID_ARG;
+  cudaPointerAttributes a;
+  cudaError_t e = cudaPointerGetAttributes(&a, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return BCJR_ERR_INVALID_ARG;
+  }
+  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return BCJR_ERR_INVALID_ARG;
+  return BCJR_OK;
+}
+
+int check_shape(int64_t n_seq, int64_t len, int L, int k, int V, Shape* sh) {
+  if (n_seq < 0 || len < 1 || k < 1 || V < 1 || L < 1) return BCJR_ERR_INVALID_ARG;
+  if (len % V != 0) return BCJR_ERR_INVALID_ARG;
+  if ((int64_t)k * V > L) return BCJR_ERR_INVALID_ARG;
+  if (L > kMaxL) return BCJR_ERR_UNSUPPORTED;
+  if (V != 1 && V != 2 && V != 4) return BCJR_ERR_UNSUPPORTED;
+  if (k * V > kMaxD) return BCJR_ERR_UNSUPPORTED;
+  if (len > kMaxLen) return BCJR_ERR_UNSUPPORTED;
+  sh->L = L; sh->k = k; sh->V = V; sh->D = k * V; sh->B = 1 << sh->D;
+  sh->J = 1 << (L - sh->D); sh->S = 1 << L; sh->n = (int)(len / V);
+  sh->n_seq = n_seq; sh->len = len;
+  return BCJR_OK;
+}
+
+int check_T(float T) { return (std::isfinite(T) && T > 0.f) ? BCJR_OK : BCJR_ERR_INVALID_ARG; }
+
+// Carves one stream-ordered allocation into 256-byte aligned pieces.
+struct Arena {
+  size_t off = 0;
+  char* base = nullptr;
+  template <class T>
+  T* take(size_t count) {
+    size_t bytes = (count * sizeof(T) + 255) & ~size_t(255);
+    T* p = reinterpret_cast<T*>(base ? base + off : nullptr);
+    off += bytes;
+    return p;
+  }
+};
+
+int threads_for(int J) {
+  int t = J < 32 ? 32 : (J > bcjr::kMaxThreads ? bcjr::kMaxThreads : J);
+  return (t + 31) / 32 * 32;
+}
+
+template <class K>
+int grid_for(K kernel, int threads, size_t smem, int64_t n_seq, int* grid) {
+  int dev = 0, nsm = 0, per = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BCJR_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return BCJR_ERR_CUDA;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return BCJR_ERR_CUDA;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kernel, threads, smem) != cudaSuccess) return BCJR_ERR_CUDA;
+  if (per < 1) return BCJR_ERR_UNSUPPORTED;
+  int64_t g = (int64_t)per * nsm;
+  if (g > n_seq) g = n_seq;
+  *grid = (int)(g < 1 ? 1 : g);
+  return BCJR_OK;
+}
+
+// ----------------------------------------------------------------- sweep
+using SweepKernel = void (*)(SweepParams);
+
+template <int MODE>
+SweepKernel pick_sweep(int V, int D) {
+#define BCJR_CASE(VV, DD) \
+  if (V == VV && D == DD) return bcjr::bcjr_sweep_kernel<VV, DD, MODE>;
+  BCJR_CASE(1, 1) BCJR_CASE(1, 2) BCJR_CASE(1, 3) BCJR_CASE(1, 4) BCJR_CASE(1, 5) BCJR_CASE(1, 6)
+  BCJR_CASE(2, 2) BCJR_CASE(2, 4) BCJR_CASE(2, 6)
+  BCJR_CASE(4, 4)
+#undef BCJR_CASE
+  return nullptr;
+}
+
+struct SweepArgs {
+  const float* w;
+  const float* c;
+  float T;
+  const float* gsoft;
+  const float* gZ;
+  float* out_soft;
+  float* out_logZ;
+  int32_t* out_argmax;
+  float* grad_w;
+  float* grad_c;
+};
+
+template <int MODE>
+int run_sweep(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
+  constexpr bool VJP = MODE == bcjr::MODE_VJP;
+  SweepKernel kern = pick_sweep<MODE>(sh.V, sh.D);
+  if (!kern) return BCJR_ERR_UNSUPPORTED;
+  const int threads = threads_for(sh.J);
+  const int NP = sh.V + 1;
+  size_t fixed = sizeof(float) * ((size_t)sh.n * sh.V * (VJP ? 2 : 1) + 64 + 64 * NP + 64 + 64);
+  size_t state_bytes = sizeof(float) * (size_t)sh.J * (VJP ? 4 : 2);
+  const bool in_smem = fixed + state_bytes <= kMaxDynSmem;
+  const size_t smem = fixed + (in_smem ? state_bytes : 0);
+  if (smem > kMaxDynSmem) return BCJR_ERR_UNSUPPORTED;
+  int grid = 0;
+  int rc = grid_for(kern, threads, smem, sh.n_seq, &grid);
+  if (rc != BCJR_OK) return rc;
+
+  const size_t SV = (size_t)sh.S * sh.V;
+  auto layout = [&](Arena& ar, SweepParams& P) {
+    P.cs = ar.take<float>(SV);
+    P.hist_l = ar.take<float>((size_t)grid * sh.n * sh.J);
+    P.hist_a = VJP ? ar.take<float>((size_t)grid * sh.n * sh.J) : nullptr;
+    P.hist_c = ar.take<double>((size_t)grid * sh.n);
+    P.state_g = in_smem ? nullptr : ar.take<float>((size_t)grid * 4 * sh.J);
+    P.gc_seq = VJP ? ar.take<float>((size_t)grid * SV) : nullptr;
+    P.gc_part = VJP ? ar.take<double>((size_t)grid * SV) : nullptr;
+  };
+  SweepParams P{};
+  Arena sizing;
+  layout(sizing, P);
+  if (fault_alloc()) return BCJR_ERR_CUDA;
+  void* mem = nullptr;
+  if (cudaMallocAsync(&mem, sizing.off, st) != cudaSuccess) {
+    cudaGetLastError();
+    return BCJR_ERR_CUDA;
+  }
+  Arena ar;
+  ar.base = static_cast<char*>(mem);
+  layout(ar, P);
+  P.w = a.w; P.gsoft = a.gsoft; P.gZ = a.gZ;
+  P.out_soft = a.out_soft; P.out_logZ = a.out_logZ; P.out_argmax = a.out_argmax; P.grad_w = a.grad_w;
+  P.n_seq = sh.n_seq; P.len = sh.len; P.L = sh.L; P.n = sh.n; P.J = sh.J; P.S = sh.S;
+  P.sk = (float)std::sqrt(1.4426950408889634 / (double)a.T);
+  P.two_over_T = (float)(2.0 / (double)a.T);
+  P.state_in_smem = in_smem ? 1 : 0;
+
+  const int sv = (int)SV;
+  bcjr::scale_codebook_kernel<<<(sv + 255) / 256, 256, 0, st>>>(a.c, sv, P.sk, const_cast<float*>(P.cs));
+  kern<<<grid, threads, smem, st>>>(P);
+  if (VJP) bcjr::reduce_gc_kernel<<<(sv + 255) / 256, 256, 0, st>>>(P.gc_part, grid, sv, a.grad_c);
+  cudaError_t le = cudaGetLastError();
+  cudaError_t fe = cudaFreeAsync(mem, st);
+  if (le != cudaSuccess || fe != cudaSuccess) return BCJR_ERR_CUDA;
+  return BCJR_OK;
+}
+
+// ----------------------------------------------------------------- Viterbi
+using ViterbiKernel = void (*)(ViterbiParams);
+
+ViterbiKernel pick_viterbi(int V, int D) {
+#define BCJR_CASE(VV, DD) \
+  if (V == VV && D == DD) return bcjr::viterbi_kernel<VV, DD>;
+  BCJR_CASE(1, 1) BCJR_CASE(1, 2) BCJR_CASE(1, 3) BCJR_CASE(1, 4) BCJR_CASE(1, 5) BCJR_CASE(1, 6)
+  BCJR_CASE(2, 2) BCJR_CASE(2, 4) BCJR_CASE(2, 6)
+  BCJR_CASE(4, 4)
+#undef BCJR_CASE
+  return nullptr;
+}
+
+int run_viterbi(const Shape& sh, const float* w, const float* c, int32_t* out_states, float* out_cost,
+                cudaStream_t st) {
+  ViterbiKernel kern = pick_viterbi(sh.V, sh.D);
+  if (!kern) return BCJR_ERR_UNSUPPORTED;
+  const int threads = threads_for(sh.J);
+  size_t fixed = sizeof(float) * ((size_t)sh.n * sh.V + 64);
+  size_t state_bytes = sizeof(float) * (size_t)sh.J * 2;
+  const bool in_smem = fixed + state_bytes <= kMaxDynSmem;
+  const size_t smem = fixed + (in_smem ? state_bytes : 0);
+  int grid = 0;
+  int rc = grid_for(kern, threads, smem, sh.n_seq, &grid);
+  if (rc != BCJR_OK) return rc;
+  ViterbiParams P{};
+  auto layout = [&](Arena& ar) {
+    P.bp = ar.take<uint8_t>((size_t)grid * sh.n * sh.J);
+    P.state_g = in_smem ? nullptr : ar.take<float>((size_t)grid * 2 * sh.J);
+  };
+  Arena sizing;
+  layout(sizing);
+  if (fault_alloc()) return BCJR_ERR_CUDA;
+  void* mem = nullptr;
+  if (cudaMallocAsync(&mem, sizing.off, st) != cudaSuccess) {
+    cudaGetLastError();
+    return BCJR_ERR_CUDA;
+  }
+  Arena ar;
+  ar.base = static_cast<char*>(mem);
+  layout(ar);
+  P.w = w; P.c = c; P.out_states = out_states; P.out_cost = out_cost;
+  P.n_seq = sh.n_seq; P.len = sh.len; P.L = sh.L; P.n = sh.n; P.J = sh.J; P.S = sh.S;
+  P.state_in_smem = in_smem ? 1 : 0;
+  kern<<<grid, threads, smem, st>>>(P);
+  cudaError_t le = cudaGetLastError();
+  cudaError_t fe = cudaFreeAsync(mem, st);
+  if (le != cudaSuccess || fe != cudaSuccess) return BCJR_ERR_CUDA;
+  return BCJR_OK;
+}
+
+__device__ int g_device_error = 0;
+
+}  // namespace
+
+extern "C" {
+
+int bcjr_soft_codeword(const float* w, int64_t n_seq, int64_t len, int L, int k, int V, const float* codebook,
+                       float T, float* out_soft, float* out_logZ, void* stream) {
+  Shape sh;
+  int rc = check_shape(n_seq, len, L, k, V, &sh);
+  if (rc) return rc;
+  if ((rc = check_T(T))) return rc;
+  if ((rc = check_dev_ptr(codebook, false))) return rc;
+  if (n_seq == 0) return BCJR_OK;
+  if ((rc = check_dev_ptr(w, false)) || (rc = check_dev_ptr(out_soft, false)) ||
+      (rc = check_dev_ptr(out_logZ, true)))
+    return rc;
+  SweepArgs a{w, codebook, T, nullptr, nullptr, out_soft, out_logZ, nullptr, nullptr, nullptr};
+  return run_sweep<bcjr::MODE_SOFT>(sh, a, static_cast<cudaStream_t>(stream));
+}
+
+int bcjr_posterior_argmax(const float* w, int64_t n_seq, int64_t len, int L, int k, int V, const float* codebook,
+                          float T, int32_t* out_argmax, void* stream) {
+  Shape sh;
+  int rc = check_shape(n_seq, len, L, k, V, &sh);
+  if (rc) return rc;
+  if ((rc = check_T(T))) return rc;
+  if ((rc = check_dev_ptr(codebook, false))) return rc;
+  if (n_seq == 0) return BCJR_OK;
+  if ((rc = check_dev_ptr(w, false)) || (rc = check_dev_ptr(out_argmax, false))) return rc;
+  SweepArgs a{w, codebook, T, nullptr, nullptr, nullptr, nullptr, out_argmax, nullptr, nullptr};
+  return run_sweep<bcjr::MODE_SOFT>(sh, a, static_cast<cudaStream_t>(stream));
+}
+
+int bcjr_vjp(const float* w, int64_t n_seq, int64_t len, int L, int k, int V, const float* codebook, float T,
+             const float* grad_soft, const float* grad_logZ, float* grad_w, float* grad_codebook, void* stream) {
+  Shape sh;
+  int rc = check_shape(n_seq, len, L, k, V, &sh);
+  if (rc) return rc;
+  if ((rc = check_T(T))) return rc;
+  if ((rc = check_dev_ptr(codebook, false)) || (rc = check_dev_ptr(grad_codebook, false))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (n_seq == 0) {
+    return cudaMemsetAsync(grad_codebook, 0, sizeof(float) * (size_t)sh.S * sh.V, st) == cudaSuccess
+               ? BCJR_OK
+               : BCJR_ERR_CUDA;
+  }
+  if ((rc = check_dev_ptr(w, false)) || (rc = check_dev_ptr(grad_soft, false)) ||
+      (rc = check_dev_ptr(grad_logZ, true)) || (rc = check_dev_ptr(grad_w, false)))
+    return rc;
+  SweepArgs a{w, codebook, T, grad_soft, grad_logZ, nullptr, nullptr, nullptr, grad_w, grad_codebook};
+  return run_sweep<bcjr::MODE_VJP>(sh, a, st);
+}
+
+int viterbi_decode(const float* w, int64_t n_seq, int64_t len, int L, int k, int V, const float* codebook,
+                   int32_t* out_states, float* out_cost, void* stream) {
+  Shape sh;
+  int rc = check_shape(n_seq, len, L, k, V, &sh);
+  if (rc) return rc;
+  if ((rc = check_dev_ptr(codebook, false))) return rc;
+  if (n_seq == 0) return BCJR_OK;
+  if ((rc = check_dev_ptr(w, false)) || (rc = check_dev_ptr(out_states, false)) ||
+      (rc = check_dev_ptr(out_cost, true)))
+    return rc;
+  return run_viterbi(sh, w, codebook, out_states, out_cost, static_cast<cudaStream_t>(stream));
+}
+
+int bcjr_get_device_error(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) {
+    cudaGetLastError();
+    return BCJR_ERR_CUDA;
+  }
+  int flag = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&flag, g_device_error, sizeof(int)) != cudaSuccess) return BCJR_ERR_CUDA;
+  if (flag != 0 && cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return BCJR_ERR_CUDA;
+  return flag;
+}
+
+const char* bcjr_strerror(int status) {
+  switch (status) {
+    case BCJR_OK: return "ok";
+    case BCJR_ERR_INVALID_ARG: return "invalid argument";
+    case BCJR_ERR_UNSUPPORTED: return "unsupported configuration";
+    case BCJR_ERR_CUDA: return "CUDA error";
+    case BCJR_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+const char* bcjr_version(void) { return "0.1.0"; }
+
+}  // extern "C"

@@ -1,0 +1,137 @@
+/*
+ * bcjr.h -- C ABI of the B200 (sm_100a) BCJR forward-backward library.
+ *
+ * The operations follow "BCJR-QAT: A Differentiable Relaxation of
+ * Trellis-Coded Weight Quantization":
+ *   - Abstract: the hard Viterbi argmax of trellis-coded quantisation is
+ *     replaced by the BCJR forward-backward sum-product at temperature T; the
+ *     result is a soft codeword equal to the Boltzmann expectation over trellis
+ *     paths, exactly differentiable, and equal to the hard code as T -> 0; the
+ *     computation is the transfer-matrix computation of a 1D Ising-like chain.
+ *   - Technical Summary, "Core Mechanism": the soft codeword
+ *       w_hat_t(T) = sum_s c(s) p_T(s_t = s | w),
+ *     differentiable in the weights and in the trellis parameters (codebook).
+ *   - Technical Summary, "Key Technical Innovations": exact gradients through
+ *     the forward-backward recursion; a fused kernel of gather, log-sum-exp and
+ *     addition.
+ *
+ * Trellis and energy (the pages leave them open; these are the readings used):
+ *   states s in [0, 2^L); D = k*V bits enter per step at the bottom:
+ *   succ(p, b) = ((p << D) & (2^L - 1)) | b, b in [0, 2^D);
+ *   step t (0 <= t < n, n = len / V) reads weights w[t*V .. t*V+V-1];
+ *   E_t(s) = sum_v (w[t*V+v] - c[s][v])^2; a path has weight exp(-sum_t E_t/T);
+ *   free start (every state has weight 1 at t = 0) and free end.
+ *
+ * Conventions for every entry point:
+ *   - All array arguments are DEVICE pointers (cudaMalloc'd or managed memory)
+ *     to contiguous row-major fp32 / int32 data, 4-byte aligned.  The caller
+ *     owns every buffer; the library never frees or retains them.
+ *   - `len` counts weights per sequence and must be a positive multiple of V.
+ *   - `codebook` is [2^L][V] fp32.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Calls are asynchronous: they validate their arguments, enqueue
+ *     the work on `stream` and return.  Argument errors are returned at once and
+ *     enqueue nothing.  The library allocates its own scratch space with
+ *     cudaMallocAsync on `stream` and frees it on `stream` before returning;
+ *     it keeps no state between calls.
+ *   - Supported: 1 <= D = k*V <= L <= 16, D <= 6, V in {1, 2, 4},
+ *     len <= 8192; T finite and > 0.  n_seq == 0 is a no-op returning BCJR_OK.
+ *   - Errors: null or non-device pointers, len not a positive multiple of V,
+ *     k < 1, V < 1, D > L, T not finite or <= 0  -> BCJR_ERR_INVALID_ARG;
+ *     L > 16, D > 6, V not in {1,2,4}, len > 8192 -> BCJR_ERR_UNSUPPORTED;
+ *     a failed CUDA call (allocation, launch)   -> BCJR_ERR_CUDA.
+ *   - NaN or infinite weights make that sequence's outputs NaN; other
+ *     sequences are unaffected.
+ */
+#ifndef BCJR_H_
+#define BCJR_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BCJR_API __attribute__((visibility("default")))
+#else
+#define BCJR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BCJR_OK = 0,
+  BCJR_ERR_INVALID_ARG = 1,
+  BCJR_ERR_UNSUPPORTED = 2,
+  BCJR_ERR_CUDA = 3,
+  BCJR_ERR_TIMEOUT = 4
+} bcjr_status;
+
+/*
+ * Soft codeword and log-partition function (Abstract; "Core Mechanism").
+ *   w         [n_seq][len]  weights (input)
+ *   codebook  [2^L][V]      codewords c(s) (input)
+ *   T                       temperature
+ *   out_soft  [n_seq][len]  w_hat: out_soft[q][t*V+v] = sum_s c(s)[v] p_t(s)
+ *   out_logZ  [n_seq]       natural log of Z = sum over paths of exp(-E/T);
+ *                           may be NULL
+ */
+BCJR_API int bcjr_soft_codeword(const float* w, int64_t n_seq, int64_t len, int L, int k, int V,
+                       const float* codebook, float T, float* out_soft, float* out_logZ, void* stream);
+
+/*
+ * Vector-Jacobian product of  l = sum_{q,t,v} grad_soft[q][t*V+v] * w_hat[q][t*V+v]
+ *                               + sum_q grad_logZ[q] * logZ[q]
+ * with respect to the weights and the codebook ("Core Mechanism": exactly
+ * differentiable with respect to the weight pre-image and the trellis
+ * parameters; "Key Technical Innovations": exact gradients).
+ *   grad_soft     [n_seq][len]  upstream gradient on out_soft (input)
+ *   grad_logZ     [n_seq]       upstream gradient on out_logZ, or NULL (= 0)
+ *   grad_w        [n_seq][len]  dl/dw (output, overwritten)
+ *   grad_codebook [2^L][V]      dl/dc summed over all sequences and steps
+ *                               (output, overwritten, not accumulated)
+ */
+BCJR_API int bcjr_vjp(const float* w, int64_t n_seq, int64_t len, int L, int k, int V, const float* codebook,
+             float T, const float* grad_soft, const float* grad_logZ, float* grad_w,
+             float* grad_codebook, void* stream);
+
+/*
+ * Viterbi decode, the T -> 0 limit of the soft codeword (Abstract: "recovering
+ * the hard QTIP code as T -> 0").  Min-sum over paths in fp32 with this exact
+ * operation order (no fused multiply-add):
+ *   q_t(s) = sum over v, in order, of fl(fl(w - c(s)[v])^2);
+ *   delta_0(s) = q_0(s);  delta_t(s) = fl(min_{p -> s} delta_{t-1}(p) + q_t(s)).
+ * Ties go to the lowest predecessor and, for the final state, the lowest index.
+ *   out_states [n_seq][n] int32   decoded state s_t of every step
+ *   out_cost   [n_seq] fp32       delta_{n-1}(s_{n-1}), or NULL
+ * T plays no part.
+ */
+BCJR_API int viterbi_decode(const float* w, int64_t n_seq, int64_t len, int L, int k, int V, const float* codebook,
+                   int32_t* out_states, float* out_cost, void* stream);
+
+/*
+ * Per-step argmax of the posterior p_T(s_t = s | w) ("Core Mechanism"), ties to
+ * the lowest state (compared in fp32).
+ *   out_argmax [n_seq][n] int32
+ */
+BCJR_API int bcjr_posterior_argmax(const float* w, int64_t n_seq, int64_t len, int L, int k, int V,
+                          const float* codebook, float T, int32_t* out_argmax, void* stream);
+
+/*
+ * Synchronises `stream` and returns BCJR_OK, or BCJR_ERR_CUDA if the stream
+ * holds a CUDA error, or the first device-side error recorded by a kernel of
+ * this library since the last call (BCJR_ERR_TIMEOUT for a bounded wait that
+ * ran out).  Reading the flag clears it.
+ */
+BCJR_API int bcjr_get_device_error(void* stream);
+
+/* Static string for a status code. */
+BCJR_API const char* bcjr_strerror(int status);
+
+/* Library version, e.g. "0.1.0". */
+BCJR_API const char* bcjr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BCJR_H_ */

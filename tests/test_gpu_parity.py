@@ -1,0 +1,150 @@
+"""GPU (C-ABI) vs CPU oracle, element by element, on small seeded cases that
+span several thread tiles, ragged sequence counts, n = 1, D = L and both V.
+
+Every call goes through libbcjr.so (include/bcjr.h) via the ctypes binding.
+"""
+import ctypes
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bcjr_sum_product_b200 import inputs as I
+from bcjr_sum_product_b200 import lib
+from helpers import assert_grad, assert_logZ, assert_soft, unique_argmax_mask
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _run_all(w, c, L, k, V, T, g, gZ):
+    wd, cd, gd, gzd = (x.to(DEV).contiguous() for x in (w, c, g, gZ))
+    soft, logZ = lib.soft_codeword(wd, cd, L, k, V, T)
+    gw, gc = lib.vjp(wd, cd, L, k, V, T, gd, gzd)
+    am = lib.posterior_argmax(wd, cd, L, k, V, T)
+    st, cost = lib.viterbi_decode(wd, cd, L, k, V)
+    torch.cuda.synchronize()
+    assert lib.get_device_error() == 0
+    return {k2: v.cpu().numpy() for k2, v in dict(soft=soft, logZ=logZ, gw=gw, gc=gc, am=am, st=st, cost=cost).items()}
+
+
+def _compare(w, c, L, k, V, T, g, gZ, gpu):
+    n = w.shape[1] // V
+    D = k * V
+    ref = oracle.soft(w, c, L, k, V, T)
+    assert_logZ(gpu["logZ"], ref["logZ"], L, D, n)
+    assert_soft(gpu["soft"], ref["soft"], c)
+    rv = oracle.vjp(w, c, L, k, V, T, g, gZ)
+    assert_grad(gpu["gw"], rv["grad_w"], "grad_w")
+    assert_grad(gpu["gc"].reshape(rv["grad_c"].shape), rv["grad_c"], "grad_c")
+    mask = unique_argmax_mask(ref["top2"])
+    np.testing.assert_array_equal(gpu["am"][mask], ref["argmax"][mask])
+    vt = oracle.viterbi(w, c, L, k, V)
+    np.testing.assert_array_equal(gpu["st"], vt["states"])
+    np.testing.assert_array_equal(gpu["cost"], vt["cost"])
+
+
+def test_tiny_workload():
+    """L=8, k=2, V=1, 16 x 64, T=0.5: soft codeword, logZ, VJP, argmax, Viterbi."""
+    inp = I.make("tiny")
+    gZ = torch.zeros(inp.w.shape[0])
+    gpu = _run_all(inp.w, inp.c, 8, 2, 1, 0.5, inp.g, gZ)
+    _compare(inp.w, inp.c, 8, 2, 1, 0.5, inp.g, gZ, gpu)
+
+
+def test_tiny_prefix_golden():
+    with open(os.path.join(os.path.dirname(__file__), "golden", "tiny_prefix6.json")) as f:
+        gold = json.load(f)
+    inp = I.make("tiny")
+    w6 = inp.w[:, :6].contiguous().to(DEV)
+    soft, logZ = lib.soft_codeword(w6, inp.c.to(DEV), 8, 2, 1, 0.5)
+    assert_logZ(logZ.cpu().numpy(), gold["logZ"], 8, 2, 6)
+    assert_soft(soft.cpu().numpy(), np.array(gold["soft"]), inp.c)
+
+
+CASES = [
+    # L, k, V, n_seq, n, T
+    (4, 2, 1, 37, 9, 0.7),
+    (4, 1, 2, 5, 6, 0.3),
+    (5, 1, 1, 33, 17, 1.3),
+    (6, 3, 2, 7, 5, 0.2),
+    (6, 6, 1, 3, 8, 0.5),      # D = L: independent softmax per step
+    (4, 4, 1, 3, 5, 0.4),      # D = L
+    (8, 2, 1, 50, 40, 0.05),
+    (10, 2, 1, 20, 64, 0.1),
+    (12, 2, 2, 6, 32, 0.05),
+    (6, 2, 1, 3, 1, 0.5),      # a single step
+    (7, 1, 1, 9, 3, 2.0),
+    (9, 2, 2, 11, 7, 0.01),    # low temperature
+    (16, 2, 1, 2, 12, 0.05),   # 65536 states, short
+    (16, 4, 2, 2, 6, 0.05),    # 65536 states, 16 branches
+]
+
+
+@pytest.mark.parametrize("L,k,V,n_seq,n,T", CASES)
+def test_random_cases(L, k, V, n_seq, n, T):
+    w, c, g = I.random_case(L, k, V, n_seq, n * V, seed=1000 + 31 * L + 7 * n + V)
+    gZ = torch.randn(n_seq, generator=torch.Generator().manual_seed(5))
+    gpu = _run_all(w, c, L, k, V, T, g, gZ)
+    _compare(w, c, L, k, V, T, g, gZ, gpu)
+
+
+def test_empty_sequence_count_is_noop_and_zeroes_codebook_gradient():
+    c = torch.randn(256, device=DEV)
+    w = torch.zeros((0, 64), device=DEV)
+    soft, logZ = lib.soft_codeword(w, c, 8, 2, 1, 0.5)
+    gc = torch.full_like(c, 7.0)
+    gw, gc = lib.vjp(w, c, 8, 2, 1, 0.5, torch.zeros_like(w), grad_codebook=gc)
+    torch.cuda.synchronize()
+    assert soft.numel() == 0 and float(gc.abs().max()) == 0.0
+
+
+def test_nan_sequence_is_isolated():
+    w, c, g = I.random_case(8, 2, 1, 5, 32, seed=77)
+    w[2, 5] = float("nan")
+    soft, logZ = lib.soft_codeword(w.to(DEV), c.to(DEV), 8, 2, 1, 0.3)
+    soft, logZ = soft.cpu().numpy(), logZ.cpu().numpy()
+    assert np.isnan(logZ[2]) and np.isnan(soft[2]).any()
+    ok = [0, 1, 3, 4]
+    ref = oracle.soft(w[ok], c, 8, 2, 1, 0.3)
+    assert_logZ(logZ[ok], ref["logZ"], 8, 2, 32)
+    assert_soft(soft[ok], ref["soft"], c)
+
+
+def test_runs_are_bit_identical():
+    w, c, g = I.random_case(12, 2, 1, 40, 64, seed=88)
+    wd, cd, gd = w.to(DEV), c.to(DEV), g.to(DEV)
+    a = lib.soft_codeword(wd, cd, 12, 2, 1, 0.1)
+    b = lib.soft_codeword(wd, cd, 12, 2, 1, 0.1)
+    ga = lib.vjp(wd, cd, 12, 2, 1, 0.1, gd)
+    gb = lib.vjp(wd, cd, 12, 2, 1, 0.1, gd)
+    for x, y in zip(a + ga, b + gb):
+        assert torch.equal(x, y)
+
+
+def test_invalid_pointers_rejected():
+    L = lib.load()
+    host = np.zeros(64, np.float32)
+    cd = torch.randn(256, device=DEV)
+    out = torch.empty((1, 64), device=DEV)
+    rc = L.bcjr_soft_codeword(host.ctypes.data_as(ctypes.c_void_p), 1, 64, 8, 2, 1,
+                              ctypes.c_void_p(cd.data_ptr()), 0.5, ctypes.c_void_p(out.data_ptr()), None, None)
+    assert rc == lib.BCJR_ERR_INVALID_ARG
+    rc = L.bcjr_soft_codeword(ctypes.c_void_p(out.data_ptr() + 2), 1, 64, 8, 2, 1,
+                              ctypes.c_void_p(cd.data_ptr()), 0.5, ctypes.c_void_p(out.data_ptr()), None, None)
+    assert rc == lib.BCJR_ERR_INVALID_ARG
+
+
+def test_forced_allocation_failure(monkeypatch):
+    w, c, g = I.random_case(8, 2, 1, 2, 16, seed=3)
+    monkeypatch.setenv("BCJR_FAULT_ALLOC", "1")
+    with pytest.raises(lib.BcjrError) as e:
+        lib.soft_codeword(w.to(DEV), c.to(DEV), 8, 2, 1, 0.5)
+    assert e.value.status == lib.BCJR_ERR_CUDA
+    monkeypatch.delenv("BCJR_FAULT_ALLOC")
+    lib.soft_codeword(w.to(DEV), c.to(DEV), 8, 2, 1, 0.5)
+    torch.cuda.synchronize()
