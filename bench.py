@@ -1,0 +1,327 @@
+#!/usr/bin/env python
+"""Throughput of the BCJR forward-backward hot path on B200.
+
+One step = one full pass of the path over one batch: ``bcjr_soft_codeword``
+(forward + backward sweep: soft codeword and logZ) followed by ``bcjr_vjp``
+(forward + backward expectation-semiring sweep: gradients w.r.t. weights and
+codebook) on the QTIP-scale workload: L=16 (65536 states), k=2, V=1, a
+2048x2048 fp32 matrix cut into 16384 sequences of 256 weights, T=0.05,
+synthetic seeded inputs (codebook seed 0, weights seed 1, upstream gradient
+seed 2).  Metric: state-updates/s = n_seq * n_steps * 2^L per step / time
+(weights/s reported alongside).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torch.distributed.run, one rank per GPU, each rank on its own
+copy of the workload (weak scaling); the codebook gradient is summed across
+ranks with one NCCL all-reduce per step.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "BCJR state-updates/s and weights/s (fwd+bwd+VJP) at L=16 k=2, 1 B200"
+UNIT = "state-updates/s"
+WORKLOAD = "qtip"
+
+# Algorithmic work per (sequence, step, state) unit for k=2, V=1 (B = 4),
+# fixed before optimisation (FP32-pipe ops, MUFU ex2 ops); recomputation and
+# ALU-pipe work (max, compares, address arithmetic) are not counted.
+LEDGER = {
+    "soft": {"fp32": 3.75 + 6.75, "mufu": 2.0},
+    "vjp": {"fp32": 7.5 + 16.5, "mufu": 2.0},
+}
+FP32_PER_CLK_SM = 128.0   # FFMA lanes per SM per clock (measured 123.5 FFMA, 126 FFMA2 on this machine)
+MUFU_PER_CLK_SM = 16.0    # ex2 per SM per clock (measured 15.99 on this machine)
+N_SM = 148
+
+
+def peak_units_per_s(kind: str, mhz: float) -> float:
+    led = LEDGER[kind] if kind != "step" else {
+        "fp32": LEDGER["soft"]["fp32"] + LEDGER["vjp"]["fp32"], "mufu": LEDGER["soft"]["mufu"] + LEDGER["vjp"]["mufu"]}
+    clk_per_unit = max(led["fp32"] / FP32_PER_CLK_SM, led["mufu"] / MUFU_PER_CLK_SM)
+    return N_SM * mhz * 1e6 / clk_per_unit
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_baseline(wl, inp, n_rows: int):
+    """The oracle as it stands, on n_rows sequences of the workload, all host cores."""
+    import oracle
+    cores = os.cpu_count() or 1
+    rows = list(range(n_rows))
+    w, g = inp.w[rows].contiguous(), inp.g[rows].contiguous()
+    T = wl.temps[0]
+    t0 = time.perf_counter()
+    oracle.soft(w, inp.c, wl.L, wl.k, wl.V, T, nthreads=cores)
+    oracle.vjp(w, inp.c, wl.L, wl.k, wl.V, T, g, nthreads=cores)
+    dt = time.perf_counter() - t0
+    units = n_rows * wl.n_steps * wl.S
+    return {"value": units / dt, "unit": UNIT, "cores": min(cores, n_rows), "kind": "oracle",
+            "sample": f"{n_rows} of {wl.n_seq} sequences of the {wl.name} workload, soft codeword + VJP, "
+                      f"fp64 C oracle with OpenMP over sequences; {dt:.1f} s"}
+
+
+def run_reference(args):
+    """The oracle arm: rank 0 times the CPU oracle on a bounded sample per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from bcjr_sum_product_b200 import inputs as I
+    wl = I.WORKLOADS[WORKLOAD]
+    cores = os.cpu_count() or 1
+    n_rows = max(1, min(cores, 16))
+    inp = I.make(WORKLOAD, rows=list(range(n_rows)))
+    import oracle
+    T = wl.temps[0]
+
+    def step():
+        oracle.soft(inp.w, inp.c, wl.L, wl.k, wl.V, T, nthreads=cores)
+        oracle.vjp(inp.w, inp.c, wl.L, wl.k, wl.V, T, inp.g, nthreads=cores)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / max(1, args.steps)
+    units = n_rows * wl.n_steps * wl.S
+    value = units / dt
+    sample = f"{n_rows} of {wl.n_seq} sequences of the {wl.name} workload per step (soft codeword + VJP)"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{wl.name}: L=16 k=2 V=1, 2048x2048 fp32 matrix as {wl.n_seq} x 256-weight "
+                                   f"sequences, T=0.05, soft codeword + logZ + VJP", "sample_sequences": n_rows},
+            "weights_per_s": n_rows * wl.seq_len / dt,
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(cores, n_rows), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    from bcjr_sum_product_b200 import inputs as I
+    from bcjr_sum_product_b200 import lib
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    lib.load()
+
+    wl = I.WORKLOADS[WORKLOAD]
+    inp = I.make(WORKLOAD)
+    T = wl.temps[0]
+    L, k, V = wl.L, wl.k, wl.V
+    stream = torch.cuda.current_stream(dev)
+    w = inp.w.to(dev); c = inp.c.to(dev); g = inp.g.to(dev)
+    soft = torch.empty_like(w); logZ = torch.empty(wl.n_seq, device=dev)
+    gw = torch.empty_like(w); gc = torch.empty_like(c)
+    flush = torch.empty(256 * 1024 * 1024 // 4, device=dev)  # 256 MB > 126 MB L2
+
+    def step():
+        lib.soft_codeword(w, c, L, k, V, T, out_soft=soft, out_logZ=logZ, stream=stream)
+        lib.vjp(w, c, L, k, V, T, g, grad_w=gw, grad_codebook=gc, stream=stream)
+        if world > 1:
+            dist.all_reduce(gc)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    soft_ms, vjp_ms, step_ms = [], [], []
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    wall0 = time.perf_counter()
+    for _ in range(args.steps):
+        flush.fill_(1.0)  # L2 flush between timed iterations (outside the events)
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record(stream)
+        lib.soft_codeword(w, c, L, k, V, T, out_soft=soft, out_logZ=logZ, stream=stream)
+        e1.record(stream)
+        lib.vjp(w, c, L, k, V, T, g, grad_w=gw, grad_codebook=gc, stream=stream)
+        if world > 1:
+            dist.all_reduce(gc)
+        e2.record(stream)
+        e2.synchronize()
+        soft_ms.append(e0.elapsed_time(e1)); vjp_ms.append(e1.elapsed_time(e2)); step_ms.append(e0.elapsed_time(e2))
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop()
+    assert lib.get_device_error(stream) == 0
+
+    total = torch.tensor([sum(step_ms), sum(soft_ms), sum(vjp_ms)], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(total, op=dist.ReduceOp.MAX)
+    ms_step = float(total[0]) / args.steps
+    ms_soft = float(total[1]) / args.steps
+    ms_vjp = float(total[2]) / args.steps
+    units = wl.units
+    value = world * units / (ms_step / 1e3)
+
+    # e2e: through the public API with host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        hw = inp.w.pin_memory(); hc = inp.c.pin_memory(); hg = inp.g.pin_memory()
+        out_soft_h = torch.empty_like(hw).pin_memory(); out_logZ_h = torch.empty(wl.n_seq).pin_memory()
+        out_gw_h = torch.empty_like(hw).pin_memory(); out_gc_h = torch.empty_like(hc).pin_memory()
+        h2d = hw.numel() * 4 + hc.numel() * 4 + hg.numel() * 4
+        d2h = out_soft_h.numel() * 4 + out_logZ_h.numel() * 4 + out_gw_h.numel() * 4 + out_gc_h.numel() * 4
+        k_e2e = max(1, min(args.steps, 3))
+        times = []
+        for _ in range(k_e2e):
+            flush.fill_(1.0)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            w.copy_(hw, non_blocking=True); c.copy_(hc, non_blocking=True); g.copy_(hg, non_blocking=True)
+            lib.soft_codeword(w, c, L, k, V, T, out_soft=soft, out_logZ=logZ, stream=stream)
+            lib.vjp(w, c, L, k, V, T, g, grad_w=gw, grad_codebook=gc, stream=stream)
+            if world > 1:
+                dist.all_reduce(gc)
+            out_soft_h.copy_(soft, non_blocking=True); out_logZ_h.copy_(logZ, non_blocking=True)
+            out_gw_h.copy_(gw, non_blocking=True); out_gc_h.copy_(gc, non_blocking=True)
+            b.record(stream)
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+        te = torch.tensor([sum(times) / len(times)], device=dev, dtype=torch.float64)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * units / (float(te[0]) / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": float(te[0])}
+
+    if rank != 0:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
+
+    peaks, basis = measured_peaks()
+    fmax = float(peaks.get("sm_max_mhz", 1965.0))
+    dominant = "vjp" if ms_vjp >= ms_soft else "soft"
+    ms_dom = ms_vjp if dominant == "vjp" else ms_soft
+    achieved = units / (ms_dom / 1e3)
+    peak = peak_units_per_s(dominant, fmax)
+    roofline = {"bound": "alu", "kernel": f"bcjr_sweep_kernel ({dominant})", "achieved": achieved, "peak": peak,
+                "unit": UNIT, "frac": achieved / peak, "traffic": None,
+                "peak_basis": f"{N_SM} SMs x min(128 FP32 / {LEDGER[dominant]['fp32']}, 16 MUFU / "
+                              f"{LEDGER[dominant]['mufu']}) units/clk at sm_max {fmax:.0f} MHz ({basis})",
+                "step_frac": value / world / peak_units_per_s("step", fmax)}
+    if clocks.get("sm_mhz"):
+        roofline["frac_at_sampled_clock"] = achieved / peak_units_per_s(dominant, clocks["sm_mhz"])
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cores = os.cpu_count() or 1
+        cpu = cpu_baseline(wl, inp, max(1, min(cores, 16)))
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"{wl.name}: L=16 k=2 V=1, 2048x2048 fp32 matrix as {wl.n_seq} x 256-weight "
+                                   f"sequences, T=0.05, soft codeword + logZ + VJP per step",
+                       "n_seq_per_gpu": wl.n_seq, "steps_per_seq": wl.n_steps, "states": wl.S,
+                       "l2": "flushed between timed iterations (256 MB write outside the events)",
+                       "parallelism": f"dp{world}" if world > 1 else "single"},
+            "weights_per_s": world * wl.n_seq * wl.seq_len / (ms_step / 1e3),
+            "ms_soft": ms_soft, "ms_vjp": ms_vjp, "wall_s": wall,
+            "gpu_launches": 5 * args.steps,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
