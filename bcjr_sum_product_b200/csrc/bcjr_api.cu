@@ -4,6 +4,7 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include <cuda_runtime.h>
 
@@ -318,3 +319,99 @@ const char* bcjr_strerror(int status) {
 const char* bcjr_version(void) { return "0.1.0"; }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------- no-allocation variant
+// bcjr_soft_codeword_noalloc: the soft-codeword sweep with its scratch taken from
+// a fixed, file-scope device array instead of cudaMallocAsync.  For callers that
+// may not allocate device memory themselves (see include/bcjr.h).
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[BCJR_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once per
+// device (the symbol name is only a host-side handle; it is not a device address).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return BCJR_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return BCJR_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return BCJR_OK;
+}
+
+}  // namespace
+
+extern "C" int bcjr_soft_codeword_noalloc(const float* w, int64_t n_seq, int64_t len, int L, int k, int V,
+                                          const float* codebook, float T, float* out_soft, float* out_logZ,
+                                          void* stream) {
+  Shape sh;
+  int rc = check_shape(n_seq, len, L, k, V, &sh);
+  if (rc) return rc;
+  if ((rc = check_T(T))) return rc;
+  if ((rc = check_dev_ptr(codebook, false))) return rc;
+  if (n_seq == 0) return BCJR_OK;
+  if ((rc = check_dev_ptr(w, false)) || (rc = check_dev_ptr(out_soft, false)) ||
+      (rc = check_dev_ptr(out_logZ, true)))
+    return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SweepKernel kern = pick_sweep<bcjr::MODE_SOFT>(sh.V, sh.D);
+  if (!kern) return BCJR_ERR_UNSUPPORTED;
+  const int threads = threads_for(sh.J);
+  const int NP = sh.V + 1;
+  const size_t fixed = sizeof(float) * ((size_t)sh.n * sh.V + 64 + 64 * NP + 64 + 64);
+  const size_t state_bytes = sizeof(float) * (size_t)sh.J * 2;
+  const bool in_smem = fixed + state_bytes <= kMaxDynSmem;
+  const size_t smem = fixed + (in_smem ? state_bytes : 0);
+  int grid = 0;
+  if ((rc = grid_for(kern, threads, smem, sh.n_seq, &grid))) return rc;
+
+  const size_t SV = (size_t)sh.S * sh.V;
+  SweepParams P{};
+  auto layout = [&](Arena& ar, int g) {
+    P.cs = ar.take<float>(SV);
+    P.hist_l = ar.take<float>((size_t)g * sh.n * sh.J);
+    P.hist_a = nullptr;
+    P.hist_c = ar.take<double>((size_t)g * sh.n);
+    P.state_g = in_smem ? nullptr : ar.take<float>((size_t)g * 4 * sh.J);
+    P.gc_seq = nullptr;
+    P.gc_part = nullptr;
+  };
+  // Fewer CTAs when the fixed scratch cannot hold one history per resident CTA.
+  for (;;) {
+    Arena sizing;
+    layout(sizing, grid);
+    if (sizing.off <= (size_t)BCJR_NOALLOC_SCRATCH_BYTES) break;
+    if (grid == 1) return BCJR_ERR_UNSUPPORTED;  // one sequence's scratch exceeds the array
+    grid = grid / 2 > 0 ? grid / 2 : 1;
+  }
+  void* base = nullptr;
+  if ((rc = noalloc_scratch(&base))) return rc;
+  Arena ar;
+  ar.base = static_cast<char*>(base);
+  layout(ar, grid);
+  P.w = w; P.gsoft = nullptr; P.gZ = nullptr;
+  P.out_soft = out_soft; P.out_logZ = out_logZ; P.out_argmax = nullptr; P.grad_w = nullptr;
+  P.n_seq = sh.n_seq; P.len = sh.len; P.L = sh.L; P.n = sh.n; P.J = sh.J; P.S = sh.S;
+  P.sk = (float)std::sqrt(1.4426950408889634 / (double)T);
+  P.two_over_T = (float)(2.0 / (double)T);
+  P.state_in_smem = in_smem ? 1 : 0;
+  const int sv = (int)SV;
+  bcjr::scale_codebook_kernel<<<(sv + 255) / 256, 256, 0, st>>>(codebook, sv, P.sk, const_cast<float*>(P.cs));
+  kern<<<grid, threads, smem, st>>>(P);
+  return cudaGetLastError() == cudaSuccess ? BCJR_OK : BCJR_ERR_CUDA;
+}

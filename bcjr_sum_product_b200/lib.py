@@ -164,3 +164,27 @@ def posterior_argmax(w: torch.Tensor, codebook: torch.Tensor, L: int, k: int, V:
 
 def get_device_error(stream=None) -> int:
     return int(load().bcjr_get_device_error(_stream(stream)))
+
+
+def soft_codeword_noalloc(w: torch.Tensor, codebook: torch.Tensor, L: int, k: int, V: int, T: float,
+                          out_soft: Optional[torch.Tensor] = None, out_logZ: Optional[torch.Tensor] = None,
+                          stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """bcjr_soft_codeword_noalloc: as soft_codeword, but the library allocates
+    nothing (its scratch is a fixed 64 MiB device array shared by all calls on a
+    device; calls that overlap on the GPU race on it).  For callers that may not
+    allocate device memory; the output tensors are still the caller's."""
+    _dev(w, "w"); _dev(codebook, "codebook")
+    n_seq, seq_len = w.shape
+    if out_soft is None:
+        out_soft = torch.empty_like(w)
+    if out_logZ is None:
+        out_logZ = torch.empty(n_seq, device=w.device, dtype=torch.float32)
+    fn = load().bcjr_soft_codeword_noalloc
+    P = ctypes.c_void_p
+    fn.argtypes = [P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, ctypes.c_float,
+                   P, P, P]
+    fn.restype = ctypes.c_int
+    rc = fn(_ptr(w), n_seq, seq_len, L, k, V, _ptr(codebook), float(T), _ptr(out_soft), _ptr(out_logZ),
+            _stream(stream))
+    _check(rc, "bcjr_soft_codeword_noalloc")
+    return out_soft, out_logZ

@@ -117,6 +117,43 @@ BCJR_API int bcjr_posterior_argmax(const float* w, int64_t n_seq, int64_t len, i
                           const float* codebook, float T, int32_t* out_argmax, void* stream);
 
 /*
+ * bcjr_soft_codeword_noalloc -- bcjr_soft_codeword without any allocation.
+ * The paper has no counterpart to this entry point; it is an interface
+ * variant for callers that must not allocate device memory: for example a
+ * plugin inside an application or framework that owns every device
+ * allocation, a service whose device-memory budget is fixed at start-up, or a
+ * latency-critical path where an allocation could block or fail under memory
+ * pressure.
+ *
+ * Arguments, layouts, results and errors are those of bcjr_soft_codeword.
+ * The call makes no cudaMalloc, cudaMallocAsync or cudaFree call and uses no
+ * allocating library routine.  Its scratch space is one fixed array of
+ * BCJR_NOALLOC_SCRATCH_BYTES (64 MiB) in this library's device memory; every
+ * GPU that loads the library reserves it until the process exits.
+ *
+ * Limit: the array must hold the scaled codebook (2^L * V floats) plus the
+ * history of one sequence ((len/V) * 2^(L-D) floats and (len/V) doubles, plus
+ * 4 * 2^(L-D) floats when the per-sequence state does not fit in shared
+ * memory).  Larger problems return BCJR_ERR_UNSUPPORTED and enqueue nothing.
+ * When the array holds fewer histories than the GPU can run at once, fewer
+ * sequences run concurrently: slower, same results.
+ *
+ * Set-up: the first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture on the device.
+ *
+ * Sharing: all calls on a device use the same array, which keeps whatever the
+ * last call left in it (nothing in it needs to start at zero).  Calls whose
+ * GPU work overlaps -- issued on different streams, or from several host
+ * threads without ordering -- race on the array and corrupt each other's
+ * results; order them, e.g. on one stream.
+ */
+#define BCJR_NOALLOC_SCRATCH_BYTES (64u << 20)
+BCJR_API int bcjr_soft_codeword_noalloc(const float* w, int64_t n_seq, int64_t len, int L, int k, int V,
+                                        const float* codebook, float T, float* out_soft, float* out_logZ,
+                                        void* stream);
+
+/*
  * Synchronises `stream` and returns BCJR_OK, or BCJR_ERR_CUDA if the stream
  * holds a CUDA error, or the first device-side error recorded by a kernel of
  * this library since the last call (BCJR_ERR_TIMEOUT for a bounded wait that

@@ -81,7 +81,7 @@ CASES = [
     (7, 1, 1, 9, 3, 2.0),
     (9, 2, 2, 11, 7, 0.01),    # low temperature
     (16, 2, 1, 2, 12, 0.05),   # 65536 states, short
-    (16, 4, 2, 2, 6, 0.05),    # 65536 states, 16 branches
+    (16, 2, 2, 2, 6, 0.05),    # 65536 states, 16 branches
 ]
 
 
