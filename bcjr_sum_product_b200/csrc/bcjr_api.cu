@@ -10,6 +10,7 @@
 
 #include "bcjr.h"
 #include "bcjr_kernels.cuh"
+#include "bcjr_l16.cuh"
 
 namespace {
 
@@ -120,9 +121,61 @@ struct SweepArgs {
   float* grad_c;
 };
 
+// L = 16, D = 2, V = 1: the block-layout kernel of bcjr_l16.cuh.
+template <int MODE>
+int run_l16(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
+  namespace K = bcjr::l16;
+  constexpr bool VJP = MODE == bcjr::MODE_VJP;
+  auto kern = K::sweep_kernel<MODE>;
+  const size_t smem = sizeof(float) * ((size_t)2 * K::J + 64 + 2 * 32 * 2 + 64 + 64 + 4 + 2 * (size_t)sh.n);
+  if (smem > kMaxDynSmem) return BCJR_ERR_UNSUPPORTED;
+  int grid = 0;
+  int rc = grid_for(kern, K::NT, smem, sh.n_seq, &grid);
+  if (rc != BCJR_OK) return rc;
+  K::Params P{};
+  auto layout = [&](Arena& ar) {
+    P.cs_tm = ar.take<float>(K::S);
+    P.hist_l = ar.take<float>((size_t)grid * sh.n * K::J);
+    P.hist_a = VJP ? ar.take<float>((size_t)grid * sh.n * K::J) : nullptr;
+    P.hist_c = ar.take<double>((size_t)grid * sh.n);
+    P.bc_g = VJP ? ar.take<float>((size_t)grid * 2 * K::J) : nullptr;
+    P.gc_part = VJP ? ar.take<double>((size_t)grid * K::S) : nullptr;
+  };
+  Arena sizing;
+  layout(sizing);
+  if (fault_alloc()) return BCJR_ERR_CUDA;
+  void* mem = nullptr;
+  if (cudaMallocAsync(&mem, sizing.off, st) != cudaSuccess) {
+    cudaGetLastError();
+    return BCJR_ERR_CUDA;
+  }
+  Arena ar;
+  ar.base = static_cast<char*>(mem);
+  layout(ar);
+  P.w = a.w; P.gsoft = a.gsoft; P.gZ = a.gZ;
+  P.out_soft = a.out_soft; P.out_logZ = a.out_logZ; P.out_argmax = a.out_argmax; P.grad_w = a.grad_w;
+  P.n_seq = sh.n_seq; P.len = sh.len; P.n = sh.n;
+  P.sk = (float)std::sqrt(1.4426950408889634 / (double)a.T);
+  P.two_over_T = (float)(2.0 / (double)a.T);
+  K::make_block_codebook<<<K::S / 256, 256, 0, st>>>(a.c, P.sk, const_cast<float*>(P.cs_tm));
+  kern<<<grid, K::NT, smem, st>>>(P);
+  if (VJP) K::reduce_block_gc<<<K::S / 256, 256, 0, st>>>(P.gc_part, grid, a.grad_c);
+  cudaError_t le = cudaGetLastError();
+  cudaError_t fe = cudaFreeAsync(mem, st);
+  if (le != cudaSuccess || fe != cudaSuccess) return BCJR_ERR_CUDA;
+  return BCJR_OK;
+}
+
+bool use_l16(const Shape& sh) {
+  const char* e = std::getenv("BCJR_GENERIC_ONLY");
+  if (e && e[0] == '1') return false;
+  return sh.L == 16 && sh.D == 2 && sh.V == 1;
+}
+
 template <int MODE>
 int run_sweep(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   constexpr bool VJP = MODE == bcjr::MODE_VJP;
+  if (use_l16(sh)) return run_l16<MODE>(sh, a, st);
   SweepKernel kern = pick_sweep<MODE>(sh.V, sh.D);
   if (!kern) return BCJR_ERR_UNSUPPORTED;
   const int threads = threads_for(sh.J);

@@ -148,3 +148,28 @@ def test_forced_allocation_failure(monkeypatch):
     monkeypatch.delenv("BCJR_FAULT_ALLOC")
     lib.soft_codeword(w.to(DEV), c.to(DEV), 8, 2, 1, 0.5)
     torch.cuda.synchronize()
+
+
+def test_l16_block_kernel_matches_generic_kernel(monkeypatch):
+    """The specialised L=16, k=2, V=1 kernels against the generic kernels on
+    300 sequences (more than one per CTA) of 64 steps, T=0.05, with gZ."""
+    w, c, g = I.random_case(16, 2, 1, 300, 64, seed=909)
+    gZ = torch.randn(300, generator=torch.Generator().manual_seed(6))
+    wd, cd, gd, gzd = w.to(DEV), c.to(DEV), g.to(DEV), gZ.to(DEV)
+    fast = [x.cpu().numpy() for x in lib.soft_codeword(wd, cd, 16, 2, 1, 0.05) + lib.vjp(wd, cd, 16, 2, 1, 0.05, gd, gzd)]
+    am_fast = lib.posterior_argmax(wd, cd, 16, 2, 1, 0.05).cpu().numpy()
+    monkeypatch.setenv("BCJR_GENERIC_ONLY", "1")
+    gen = [x.cpu().numpy() for x in lib.soft_codeword(wd, cd, 16, 2, 1, 0.05) + lib.vjp(wd, cd, 16, 2, 1, 0.05, gd, gzd)]
+    am_gen = lib.posterior_argmax(wd, cd, 16, 2, 1, 0.05).cpu().numpy()
+    assert_soft(fast[0], gen[0], c)
+    assert_logZ(fast[1], gen[1], 16, 2, 64)
+    assert_grad(fast[2], gen[2], "grad_w")
+    assert_grad(fast[3], gen[3], "grad_c")
+    assert (am_fast == am_gen).mean() > 0.999
+    # and both against the oracle on a few rows
+    rows = [0, 147, 148, 299]
+    ref = oracle.soft(w[rows], c, 16, 2, 1, 0.05)
+    assert_logZ(fast[1][rows], ref["logZ"], 16, 2, 64)
+    assert_soft(fast[0][rows], ref["soft"], c)
+    rv = oracle.vjp(w[rows], c, 16, 2, 1, 0.05, g[rows], gZ[rows])
+    assert_grad(fast[2][rows], rv["grad_w"], "grad_w")
