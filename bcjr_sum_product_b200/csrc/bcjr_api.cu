@@ -32,6 +32,46 @@ bool fault_alloc() {
   return e && e[0] == '1';
 }
 
+// Library-private stream-ordered pool per device.  Scratch freed at the end of
+// a call stays mapped in the pool (release threshold = unlimited), so the next
+// call of the same size reuses it instead of mapping gigabytes again.
+constexpr int kMaxPoolDevices = 64;
+std::mutex g_pool_mu;
+cudaMemPool_t g_pool[kMaxPoolDevices] = {};
+
+int scratch_alloc(void** mem, size_t bytes, cudaStream_t st) {
+  if (fault_alloc()) return BCJR_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxPoolDevices) {
+    cudaGetLastError();
+    return BCJR_ERR_CUDA;
+  }
+  cudaMemPool_t pool;
+  {
+    std::lock_guard<std::mutex> lk(g_pool_mu);
+    if (g_pool[dev] == nullptr) {
+      cudaMemPoolProps props = {};
+      props.allocType = cudaMemAllocationTypePinned;
+      props.location.type = cudaMemLocationTypeDevice;
+      props.location.id = dev;
+      cudaMemPool_t p;
+      if (cudaMemPoolCreate(&p, &props) != cudaSuccess) {
+        cudaGetLastError();
+        return BCJR_ERR_CUDA;
+      }
+      uint64_t thr = UINT64_MAX;
+      cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &thr);
+      g_pool[dev] = p;
+    }
+    pool = g_pool[dev];
+  }
+  if (cudaMallocFromPoolAsync(mem, bytes, pool, st) != cudaSuccess) {
+    cudaGetLastError();
+    return BCJR_ERR_CUDA;
+  }
+  return BCJR_OK;
+}
+
 int check_dev_ptr(const void* p, bool nullable) {
   if (p == nullptr) return nullable ? BCJR_OK : BCJR_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(p) % 4 != 0) return BCJR_ERR_INVALID_ARG;
@@ -126,7 +166,8 @@ template <int MODE>
 int run_l16(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   namespace K = bcjr::l16;
   constexpr bool VJP = MODE == bcjr::MODE_VJP;
-  auto kern = K::sweep_kernel<MODE>;
+  void (*kern)(K::Params) = K::vjp_kernel;
+  if (!VJP) kern = a.out_argmax ? K::soft_kernel<true> : K::soft_kernel<false>;
   const size_t smem = sizeof(float) * ((size_t)2 * K::J + 64 + 2 * 32 * 2 + 64 + 64 + 4 + 2 * (size_t)sh.n);
   if (smem > kMaxDynSmem) return BCJR_ERR_UNSUPPORTED;
   int grid = 0;
@@ -143,12 +184,8 @@ int run_l16(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   };
   Arena sizing;
   layout(sizing);
-  if (fault_alloc()) return BCJR_ERR_CUDA;
   void* mem = nullptr;
-  if (cudaMallocAsync(&mem, sizing.off, st) != cudaSuccess) {
-    cudaGetLastError();
-    return BCJR_ERR_CUDA;
-  }
+  if (int arc = scratch_alloc(&mem, sizing.off, st)) return arc;
   Arena ar;
   ar.base = static_cast<char*>(mem);
   layout(ar);
@@ -202,12 +239,8 @@ int run_sweep(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   SweepParams P{};
   Arena sizing;
   layout(sizing, P);
-  if (fault_alloc()) return BCJR_ERR_CUDA;
   void* mem = nullptr;
-  if (cudaMallocAsync(&mem, sizing.off, st) != cudaSuccess) {
-    cudaGetLastError();
-    return BCJR_ERR_CUDA;
-  }
+  if (int arc = scratch_alloc(&mem, sizing.off, st)) return arc;
   Arena ar;
   ar.base = static_cast<char*>(mem);
   layout(ar, P);
@@ -260,12 +293,8 @@ int run_viterbi(const Shape& sh, const float* w, const float* c, int32_t* out_st
   };
   Arena sizing;
   layout(sizing);
-  if (fault_alloc()) return BCJR_ERR_CUDA;
   void* mem = nullptr;
-  if (cudaMallocAsync(&mem, sizing.off, st) != cudaSuccess) {
-    cudaGetLastError();
-    return BCJR_ERR_CUDA;
-  }
+  if (int arc = scratch_alloc(&mem, sizing.off, st)) return arc;
   Arena ar;
   ar.base = static_cast<char*>(mem);
   layout(ar);

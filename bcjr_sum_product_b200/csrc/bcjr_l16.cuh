@@ -16,12 +16,17 @@
 //   exchanged through shared memory.
 //
 //   512 threads; thread tau owns blocks mid = tau + 512 k, k = 0..7.
-//   The scaled codebook is stored block-major: cs_tm[mid * 16 + 4 h + lo], so
-//   a thread's 16 codewords of a block are one 64-byte line; it is the same
-//   every step, so the next block's line is always prefetched.
-//   VJP: the per-state codebook gradient of the current sequence lives in
-//   tensor memory (512 columns x 128 lanes = 65536 fp32 = one per state),
-//   warp w holding lanes 32 (w mod 4) .. + 31, columns 128 (w div 4) + 16 k.
+//   The scaled codebook is stored block-major, cs_tm[mid * 16 + bidx(h, lo)]
+//   with bidx(h, lo) = 8 (h >> 1) + 2 lo + (h & 1): a thread's 16 codewords of
+//   a block are one 64-byte line (the same every step), the two halves are
+//   the h-pairs {0,1} and {2,3}, and within a half the pair (2g, 2g+1) of one
+//   bottom digit lo is adjacent, feeding the packed f32x2 instructions in
+//   both directions.
+//   Tensor memory (512 columns x 128 lanes = 65536 fp32, one per state) holds,
+//   for SOFT, the thread's codewords (read back every step without touching
+//   L2) and, for VJP, the current sequence's per-state codebook gradient
+//   (the VJP streams the codebook from L2 instead); warp w uses lanes
+//   32 (w mod 4) .. + 31 and columns 128 (w div 4) + 16 k for block k.
 #pragma once
 #include "bcjr_kernels.cuh"
 
@@ -88,6 +93,25 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&r)[16]) 
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&r)[8]) {
+  uint32_t u[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7])
+               : "r"(taddr)
+               : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) r[i] = __uint_as_float(u[i]);
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+               "r"(__float_as_uint(r[0])), "r"(__float_as_uint(r[1])), "r"(__float_as_uint(r[2])),
+               "r"(__float_as_uint(r[3])), "r"(__float_as_uint(r[4])), "r"(__float_as_uint(r[5])),
+               "r"(__float_as_uint(r[6])), "r"(__float_as_uint(r[7]))
+               : "memory");
+}
+
+__host__ __device__ constexpr int bidx(int h, int lo) { return 8 * (h >> 1) + 2 * lo + (h & 1); }
 
 __device__ __forceinline__ void ld_cb(const float* __restrict__ cs_tm, int mid, float (&c)[16]) {
   const float4* p = reinterpret_cast<const float4*>(cs_tm + (size_t)mid * 16);
@@ -98,11 +122,18 @@ __device__ __forceinline__ void ld_cb(const float* __restrict__ cs_tm, int mid, 
   }
 }
 
-// c_tm[mid * 16 + 4 h + lo] = sk * c[(h << 14) | (mid << 2) | lo]
+// The half of block mid holding the h-pair g: 8 codewords, index 2 lo + (h & 1).
+__device__ __forceinline__ void ld_cb8(const float* __restrict__ cs_tm, int mid, int g, float (&c)[8]) {
+  const float4* p = reinterpret_cast<const float4*>(cs_tm + (size_t)mid * 16 + 8 * g);
+  const float4 a = __ldg(p), b = __ldg(p + 1);
+  c[0] = a.x; c[1] = a.y; c[2] = a.z; c[3] = a.w; c[4] = b.x; c[5] = b.y; c[6] = b.z; c[7] = b.w;
+}
+
+// cs_tm[mid * 16 + bidx(h, lo)] = sk * c[(h << 14) | (mid << 2) | lo]
 __global__ void make_block_codebook(const float* __restrict__ c, float sk, float* __restrict__ cs_tm) {
   int x = blockIdx.x * blockDim.x + threadIdx.x;
   if (x >= S) return;
-  const int mid = x >> 4, h = (x >> 2) & 3, lo = x & 3;
+  const int mid = x >> 4, r = x & 15, h = ((r >> 3) << 1) | (r & 1), lo = (r >> 1) & 3;
   cs_tm[x] = sk * c[(h << 14) | (mid << 2) | lo];
 }
 
@@ -111,309 +142,548 @@ __global__ void reduce_block_gc(const double* __restrict__ part, int nparts, flo
   int q = blockIdx.x * blockDim.x + threadIdx.x;
   if (q >= S) return;
   const int h = q >> 14, mid = (q >> 2) & (NMID - 1), lo = q & 3;
-  const size_t x = (size_t)mid * 16 + 4 * h + lo;
+  const size_t x = (size_t)mid * 16 + bidx(h, lo);
   double a = 0.0;
   for (int p = 0; p < nparts; ++p) a += part[(size_t)p * S + x];
   out[q] = (float)a;
 }
 
-template <int MODE>
-__global__ void __launch_bounds__(NT, 1) sweep_kernel(Params P) {
-  constexpr bool VJP = (MODE == MODE_VJP);
+// ------------------------------------------------------------ soft pass, packed
+// The soft-codeword pass (forward + backward + posterior + w_hat, optional
+// posterior argmax) with the FP32 work in packed f32x2 instructions.  Log
+// values are kept negated ("energies", n = -log2), so that each group is
+//   x'_h = d_h^2 + n_h,  m' = min_h x'_h,  n_new = m' - log2 sum_h 2^(m' - x'_h) - offset,
+// every line an FFMA/FADD without negations.  Pairs (h, h+1) share one f32x2
+// lane pair: in the forward they are two members of one group, in the
+// backward two groups with the same member.
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+__device__ __forceinline__ float2 f2s(float a) { return make_float2(a, a); }
+
+template <bool ARGMAX>
+__global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
   constexpr int NP = 2;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int nwarps = NT / 32;
   const int n = P.n;
 
   extern __shared__ __align__(16) float smem[];
-  float* sb = smem;                                    // [2][J] state ping-pong (16-byte aligned)
+  float* sb = smem;                                    // [2][J] negated state ping-pong
   float* lb[2] = {sb, sb + J};
-  float* wmax = sb + 2 * J;                            // [2][32]
-  float* part = wmax + 64;                             // [2][32][NP]
+  float* wmin = sb + 2 * J;                            // [2][32]
+  float* part = wmin + 64;                             // [2][32][NP]
   float* apart = part + 2 * 32 * NP;                   // [2][32]
   int* aidx = reinterpret_cast<int*>(apart + 64);      // [2][32]
   uint32_t* tslot = reinterpret_cast<uint32_t*>(aidx + 64);  // [4]
   float* wsc = reinterpret_cast<float*>(tslot + 4);    // n
-  float* gsc = wsc + n;                                // n (VJP)
 
-  float* hist_l = P.hist_l + (size_t)blockIdx.x * n * J;
-  float* hist_a = VJP ? P.hist_a + (size_t)blockIdx.x * n * J : nullptr;
+  float* hist = P.hist_l + (size_t)blockIdx.x * n * J;   // negated forward values
   double* hist_c = P.hist_c + (size_t)blockIdx.x * n;
-  float* bcg[2] = {nullptr, nullptr};
-  double* gcp = nullptr;
-  if constexpr (VJP) {
-    bcg[0] = P.bc_g + (size_t)blockIdx.x * 2 * J;
-    bcg[1] = bcg[0] + J;
-    gcp = P.gc_part + (size_t)blockIdx.x * S;
-  }
-  const float* __restrict__ cs_tm = P.cs_tm;
+  const float2 neg1 = f2s(-1.f);
 
-  uint32_t tbase = 0;
-  if constexpr (VJP) {
-    if (warp == 0) tmem_alloc512(tslot);
-    tmem_fence_before();
-    __syncthreads();
-    tmem_fence_after();
-    tbase = tslot[0] + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(128 * (warp >> 2));
-    float z16[16];
+  if (warp == 0) tmem_alloc512(tslot);
+  tmem_fence_before();
+  __syncthreads();
+  tmem_fence_after();
+  const uint32_t tbase = tslot[0] + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(128 * (warp >> 2));
 #pragma unroll
-    for (int i = 0; i < 16; ++i) z16[i] = 0.f;
-#pragma unroll
-    for (int k = 0; k < KB; ++k) tmem_st16(tbase + 16 * k, z16);
-    tmem_wait_st();
-    for (int x = tid; x < S; x += NT) gcp[x] = 0.0;
+  for (int k = 0; k < KB; ++k) {
+    float c16[16];
+    ld_cb(P.cs_tm, tid + NT * k, c16);
+    tmem_st16(tbase + 16 * k, c16);
   }
+  tmem_wait_st();
 
   for (int64_t seq = blockIdx.x; seq < P.n_seq; seq += gridDim.x) {
     const float* wq = P.w + seq * P.len;
-    for (int x = tid; x < n; x += NT) wsc[x] = wq[x] * P.sk;
-    if constexpr (VJP) {
-      const float* gq = P.gsoft + seq * P.len;
-      for (int x = tid; x < n; x += NT) gsc[x] = gq[x] / P.sk;
-    }
+    for (int x = tid; x < n; x += NT) wsc[x] = -wq[x] * P.sk;   // -w'
     __syncthreads();
 
-    // ---------------------------------------------------------- forward
-    float R = 0.f;
-    double C = 0.0;
-    float cbn[16];
-    ld_cb(cs_tm, tid, cbn);
+    // ------------------------------------------------------------ forward
+    float Rn = 0.f;     // min of the previous step's stored (negated) values
+    double C = 0.0;     // log2 sigma_t = -stored + C_t
     for (int t = 0; t < n; ++t) {
-      const float* lprev = lb[(t + 1) & 1];
-      float* lcur = lb[t & 1];
-      const float wt = wsc[t];
-      const float gt = VJP ? gsc[t] : 0.f;
-      const float* aprev = (VJP && t > 0) ? hist_a + (size_t)(t - 1) * J : nullptr;
-      C += (double)R;
-      float tmax = -INFINITY;
+      const float* nprev = lb[(t + 1) & 1];
+      float* ncur = lb[t & 1];
+      const float2 nw2 = f2s(wsc[t]);
+      C -= (double)Rn;
+      float tmin = INFINITY;
 #pragma unroll
       for (int k = 0; k < KB; ++k) {
         const int mid = tid + NT * k;
         float cb[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) cb[i] = cbn[i];
-        ld_cb(cs_tm, (k + 1 < KB) ? mid + NT : tid, cbn);
-        float lsp[4], asp[4];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          lsp[h] = (t == 0) ? 0.f : lprev[(h << HB) | mid];
-          if constexpr (VJP) asp[h] = (t == 0) ? 0.f : aprev[(h << HB) | mid];
+        tmem_ld16(tbase + 16 * k, cb);
+        float2 np01, np23;
+        if (t == 0) {
+          np01 = f2s(0.f); np23 = f2s(0.f);
+        } else {
+          np01 = f2(nprev[(0 << HB) | mid], nprev[(1 << HB) | mid]);
+          np23 = f2(nprev[(2 << HB) | mid], nprev[(3 << HB) | mid]);
+          // history of step t-1 in block-major order [mid][h]: what the backward reads per block
+          reinterpret_cast<float4*>(hist + (size_t)(t - 1) * J)[mid] = make_float4(np01.x, np01.y, np23.x, np23.y);
         }
-        float lout[4], aout[4];
+        float out[4];
 #pragma unroll
         for (int lo = 0; lo < 4; ++lo) {
-          float x[4];
-          float m = -INFINITY;
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const float d = wt - cb[4 * h + lo];
-            x[h] = fmaf(-d, d, lsp[h]);
-            m = fmaxf(m, x[h]);
-          }
-          float s = 0.f, num = 0.f;
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const float u = ex2f(x[h] - m);
-            s += u;
-            if constexpr (VJP) num = fmaf(u, fmaf(gt, cb[4 * h + lo], asp[h]), num);
-          }
-          lout[lo] = m + lg2f(s) - R;
-          if constexpr (VJP) aout[lo] = __fdividef(num, s);
-          tmax = fmaxf(tmax, lout[lo]);
+          const float2 d01 = __fadd2_rn(f2(cb[bidx(0, lo)], cb[bidx(1, lo)]), nw2);
+          const float2 d23 = __fadd2_rn(f2(cb[bidx(2, lo)], cb[bidx(3, lo)]), nw2);
+          const float2 x01 = __ffma2_rn(d01, d01, np01);
+          const float2 x23 = __ffma2_rn(d23, d23, np23);
+          const float m = fminf(fminf(x01.x, x01.y), fminf(x23.x, x23.y));
+          const float2 a01 = __ffma2_rn(x01, neg1, f2s(m));
+          const float2 a23 = __ffma2_rn(x23, neg1, f2s(m));
+          const float2 s2 = __fadd2_rn(f2(ex2f(a01.x), ex2f(a01.y)), f2(ex2f(a23.x), ex2f(a23.y)));
+          out[lo] = (m - Rn) - lg2f(s2.x + s2.y);
         }
-        const float4 l4 = make_float4(lout[0], lout[1], lout[2], lout[3]);
-        reinterpret_cast<float4*>(lcur)[mid] = l4;
-        if (t < n - 1) reinterpret_cast<float4*>(hist_l + (size_t)t * J)[mid] = l4;
-        if constexpr (VJP)
-          reinterpret_cast<float4*>(hist_a + (size_t)t * J)[mid] = make_float4(aout[0], aout[1], aout[2], aout[3]);
+        tmin = fminf(tmin, fminf(fminf(out[0], out[1]), fminf(out[2], out[3])));
+        reinterpret_cast<float4*>(ncur)[mid] = make_float4(out[0], out[1], out[2], out[3]);
       }
-      tmax = warp_max(tmax);
-      if (lane == 0) wmax[(t & 1) * 32 + warp] = tmax;
+      tmin = -warp_max(-tmin);
+      if (lane == 0) wmin[(t & 1) * 32 + warp] = tmin;
       if (tid == 0) hist_c[t] = C;
       __syncthreads();
-      R = -INFINITY;
+      Rn = INFINITY;
 #pragma unroll
-      for (int w2 = 0; w2 < nwarps; ++w2) R = fmaxf(R, wmax[(t & 1) * 32 + w2]);
+      for (int w2 = 0; w2 < nwarps; ++w2) Rn = fminf(Rn, wmin[(t & 1) * 32 + w2]);
+    }
+    // log2 Z = -Rn + log2 sum_j 2^(Rn - stored_j) + C
+    double l2Z;
+    {
+      const float* nfin = lb[(n - 1) & 1];
+      float s0 = 0.f;
+      for (int j = tid; j < J; j += NT) s0 += ex2f(Rn - nfin[j]);
+      s0 = warp_sum(s0);
+      if (lane == 0) part[warp * NP] = s0;
+      __syncthreads();
+      float a0 = 0.f;
+#pragma unroll
+      for (int w2 = 0; w2 < nwarps; ++w2) a0 += part[w2 * NP];
+      l2Z = -(double)Rn + log2((double)a0) + C;
+      if (tid == 0 && P.out_logZ) P.out_logZ[seq] = (float)(l2Z * 0.69314718055994530942);
+      __syncthreads();
     }
 
-    // logZ, Hbar
+    // ------------------------------------------------------------ backward
+    float Rrn = 0.f;
+    double Cr = 0.0;   // log2 beta_t = -stored + Cr_t
+    // block kk of step tt reads step tt-1's values (free start: 0 for tt = 0)
+    auto hist_at = [&](int tt, int kk) -> float4 {
+      return (tt >= 1) ? reinterpret_cast<const float4*>(hist + (size_t)(tt - 1) * J)[tid + NT * kk]
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    };
+    float4 hsn = hist_at(n - 1, 0), hsm = hist_at(n - 1, 1);
+    for (int t = n - 1; t >= 0; --t) {
+      const float* ncur = lb[t & 1];
+      float* nnext = lb[(t + 1) & 1];
+      const float2 nw2 = f2s(wsc[t]);
+      const double Csig = (t >= 1) ? hist_c[t - 1] : 0.0;
+      const float K = (float)(Csig + Cr - l2Z);
+      const bool last = (t == n - 1);
+      float2 accc = f2s(0.f), accp = f2s(0.f);
+      float bestp = -1.f;
+      int bestq = 0x7fffffff;
+      float tmin = INFINITY;
+#pragma unroll
+      for (int k = 0; k < KB; ++k) {
+        const int mid = tid + NT * k;
+        float cb[16];
+        tmem_ld16(tbase + 16 * k, cb);
+        const float hs[4] = {hsn.x, hsn.y, hsn.z, hsn.w};
+        {
+          const int nt = (k + 2 < KB) ? t : t - 1, nk = (k + 2 < KB) ? k + 2 : k + 2 - KB;
+          hsn = hsm;
+          hsm = hist_at(nt, nk);
+        }
+        float nr[4];
+        if (last) {
+          nr[0] = nr[1] = nr[2] = nr[3] = 0.f;
+        } else {
+          const float4 rv = reinterpret_cast<const float4*>(ncur)[mid];
+          nr[0] = rv.x; nr[1] = rv.y; nr[2] = rv.z; nr[3] = rv.w;
+        }
+        float nout[4];
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {          // groups h = 2g, 2g+1 side by side
+          float2 y[4];
+#pragma unroll
+          for (int lo = 0; lo < 4; ++lo) {
+            const float2 d = __fadd2_rn(f2(cb[bidx(2 * g, lo)], cb[bidx(2 * g + 1, lo)]), nw2);
+            y[lo] = __ffma2_rn(d, d, f2s(nr[lo]));
+          }
+          const float2 m = f2(fminf(fminf(y[0].x, y[1].x), fminf(y[2].x, y[3].x)),
+                              fminf(fminf(y[0].y, y[1].y), fminf(y[2].y, y[3].y)));
+          // posterior factor of each group: 2^(K - m' - n_sigma)
+          const float2 ge = __fadd2_rn(__fadd2_rn(f2s(K), f2(-hs[2 * g], -hs[2 * g + 1])), __fmul2_rn(m, neg1));
+          const float2 gf = f2(ex2f(ge.x), ex2f(ge.y));
+          float2 ssum = f2s(0.f);
+#pragma unroll
+          for (int lo = 0; lo < 4; ++lo) {
+            const float2 a = __ffma2_rn(y[lo], neg1, m);
+            const float2 u = f2(ex2f(a.x), ex2f(a.y));
+            ssum = __fadd2_rn(ssum, u);
+            const float2 pp = __fmul2_rn(u, gf);
+            accc = __ffma2_rn(pp, f2(cb[bidx(2 * g, lo)], cb[bidx(2 * g + 1, lo)]), accc);
+            accp = __fadd2_rn(accp, pp);
+            if constexpr (ARGMAX) {
+              arg_better(bestp, bestq, pp.x, ((2 * g) << 14) | (mid << 2) | lo);
+              arg_better(bestp, bestq, pp.y, ((2 * g + 1) << 14) | (mid << 2) | lo);
+            }
+          }
+          nout[2 * g] = (m.x - Rrn) - lg2f(ssum.x);
+          nout[2 * g + 1] = (m.y - Rrn) - lg2f(ssum.y);
+        }
+        if (t >= 1) {
+#pragma unroll
+          for (int h = 0; h < 4; ++h) nnext[(h << HB) | mid] = nout[h];
+          tmin = fminf(tmin, fminf(fminf(nout[0], nout[1]), fminf(nout[2], nout[3])));
+        }
+      }
+      float a0 = warp_sum(accc.x + accc.y);
+      float a1 = warp_sum(accp.x + accp.y);
+      tmin = -warp_max(-tmin);
+      if constexpr (ARGMAX) warp_argmax(bestp, bestq);
+      const int pb = t & 1;
+      if (lane == 0) {
+        part[(pb * 32 + warp) * NP] = a0;
+        part[(pb * 32 + warp) * NP + 1] = a1;
+        wmin[pb * 32 + warp] = tmin;
+        if constexpr (ARGMAX) { apart[pb * 32 + warp] = bestp; aidx[pb * 32 + warp] = bestq; }
+      }
+      __syncthreads();
+      if (tid == 0) {
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int w2 = 0; w2 < nwarps; ++w2) { s0 += part[(pb * 32 + w2) * NP]; s1 += part[(pb * 32 + w2) * NP + 1]; }
+        if (P.out_soft) P.out_soft[seq * P.len + t] = s0 / (s1 * P.sk);
+        if constexpr (ARGMAX) {
+          float bp = -1.f;
+          int bq = 0x7fffffff;
+#pragma unroll
+          for (int w2 = 0; w2 < nwarps; ++w2) arg_better(bp, bq, apart[pb * 32 + w2], aidx[pb * 32 + w2]);
+          if (P.out_argmax) P.out_argmax[seq * n + t] = bq;
+        }
+      }
+      Cr -= (double)Rrn;
+      Rrn = INFINITY;
+#pragma unroll
+      for (int w2 = 0; w2 < nwarps; ++w2) Rrn = fminf(Rrn, wmin[pb * 32 + w2]);
+    }
+    __syncthreads();
+  }
+
+  tmem_fence_before();
+  __syncthreads();
+  tmem_fence_after();
+  if (warp == 0) tmem_dealloc512(tslot[0]);
+}
+
+
+// ------------------------------------------------------------ VJP pass, packed
+// Forward (negated log sigma and the prefix expectation A), then backward
+// (negated log rho, suffix expectation Bc, G, dl/dw per step and the per-state
+// codebook gradient).  Tensor memory holds the codewords during the forward
+// and the current sequence's codebook gradient during the backward, when the
+// codewords stream from L2 (block-major lines, prefetched one block ahead).
+// The forward's A_t ping-pongs in global scratch (L2-resident); both
+// histories (negated log sigma and A) go to HBM in block-major order [mid][h],
+// written by the next forward step from the values it has just read, so that
+// the backward loads one 16-byte vector of each per block.  The backward's Bc
+// ping-pongs in the same global scratch.
+__global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
+  constexpr int NP = 2;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int nwarps = NT / 32;
+  const int n = P.n;
+
+  extern __shared__ __align__(16) float smem[];
+  float* sb = smem;                                    // [2][J] negated state ping-pong
+  float* lb[2] = {sb, sb + J};
+  float* wmin = sb + 2 * J;                            // [2][32]
+  float* part = wmin + 64;                             // [2][32][NP]
+  float* spare = part + 2 * 32 * NP;                   // [2][32] + [2][32] (unused)
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(spare + 128);  // [4]
+  float* wsc = reinterpret_cast<float*>(tslot + 4);    // n: -w'
+  float* gsc = wsc + n;                                // n: g / sk
+
+  float* hist_l = P.hist_l + (size_t)blockIdx.x * n * J;
+  float* hist_a = P.hist_a + (size_t)blockIdx.x * n * J;
+  double* hist_c = P.hist_c + (size_t)blockIdx.x * n;
+  float* bcg[2] = {P.bc_g + (size_t)blockIdx.x * 2 * J, P.bc_g + (size_t)blockIdx.x * 2 * J + J};
+  double* gcp = P.gc_part + (size_t)blockIdx.x * S;
+  const float* __restrict__ cs_tm = P.cs_tm;
+  const float2 neg1 = f2s(-1.f);
+
+  if (warp == 0) tmem_alloc512(tslot);
+  tmem_fence_before();
+  __syncthreads();
+  tmem_fence_after();
+  const uint32_t tbase = tslot[0] + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(128 * (warp >> 2));
+  for (int x = tid; x < S; x += NT) gcp[x] = 0.0;
+
+  for (int64_t seq = blockIdx.x; seq < P.n_seq; seq += gridDim.x) {
+    const float* wq = P.w + seq * P.len;
+    const float* gq = P.gsoft + seq * P.len;
+    for (int x = tid; x < n; x += NT) { wsc[x] = -wq[x] * P.sk; gsc[x] = gq[x] / P.sk; }
+    // codewords into tensor memory for the forward
+#pragma unroll
+    for (int k = 0; k < KB; ++k) {
+      float c16[16];
+      ld_cb(cs_tm, tid + NT * k, c16);
+      tmem_st16(tbase + 16 * k, c16);
+    }
+    tmem_wait_st();
+    __syncthreads();
+
+    // ------------------------------------------------------------ forward
+    float Rn = 0.f;
+    double C = 0.0;
+    for (int t = 0; t < n; ++t) {
+      const float* nprev = lb[(t + 1) & 1];
+      float* ncur = lb[t & 1];
+      // A_t ping-pongs in global scratch (L2-resident); the history copy is block-major
+      const float* aprev = bcg[(t + 1) & 1];
+      float* acur = bcg[t & 1];
+      const float2 nw2 = f2s(wsc[t]);
+      const float2 g2 = f2s(gsc[t]);
+      C -= (double)Rn;
+      float tmin = INFINITY;
+      float apn[4] = {0.f, 0.f, 0.f, 0.f};
+      if (t > 0) {
+#pragma unroll
+        for (int h = 0; h < 4; ++h) apn[h] = aprev[(h << HB) | tid];
+      }
+#pragma unroll
+      for (int k = 0; k < KB; ++k) {
+        const int mid = tid + NT * k;
+        float cb[16];
+        tmem_ld16(tbase + 16 * k, cb);
+        const float2 ap01 = f2(apn[0], apn[1]), ap23 = f2(apn[2], apn[3]);
+        if (t > 0 && k + 1 < KB) {
+#pragma unroll
+          for (int h = 0; h < 4; ++h) apn[h] = aprev[(h << HB) | (mid + NT)];
+        }
+        float2 np01, np23;
+        if (t == 0) {
+          np01 = f2s(0.f); np23 = f2s(0.f);
+        } else {
+          np01 = f2(nprev[(0 << HB) | mid], nprev[(1 << HB) | mid]);
+          np23 = f2(nprev[(2 << HB) | mid], nprev[(3 << HB) | mid]);
+          // step t-1's values in block-major order [mid][h], as the backward reads them
+          reinterpret_cast<float4*>(hist_l + (size_t)(t - 1) * J)[mid] = make_float4(np01.x, np01.y, np23.x, np23.y);
+          reinterpret_cast<float4*>(hist_a + (size_t)(t - 1) * J)[mid] = make_float4(ap01.x, ap01.y, ap23.x, ap23.y);
+        }
+        float out[4], aout[4];
+#pragma unroll
+        for (int lo = 0; lo < 4; ++lo) {
+          const float2 c01 = f2(cb[bidx(0, lo)], cb[bidx(1, lo)]), c23 = f2(cb[bidx(2, lo)], cb[bidx(3, lo)]);
+          const float2 d01 = __fadd2_rn(c01, nw2), d23 = __fadd2_rn(c23, nw2);
+          const float2 x01 = __ffma2_rn(d01, d01, np01), x23 = __ffma2_rn(d23, d23, np23);
+          const float m = fminf(fminf(x01.x, x01.y), fminf(x23.x, x23.y));
+          const float2 a01 = __ffma2_rn(x01, neg1, f2s(m)), a23 = __ffma2_rn(x23, neg1, f2s(m));
+          const float2 u01 = f2(ex2f(a01.x), ex2f(a01.y)), u23 = f2(ex2f(a23.x), ex2f(a23.y));
+          const float2 z01 = __ffma2_rn(g2, c01, ap01), z23 = __ffma2_rn(g2, c23, ap23);
+          const float2 s2 = __fadd2_rn(u01, u23);
+          const float2 q2 = __ffma2_rn(u23, z23, __fmul2_rn(u01, z01));
+          const float ssum = s2.x + s2.y;
+          out[lo] = (m - Rn) - lg2f(ssum);
+          aout[lo] = __fdividef(q2.x + q2.y, ssum);
+        }
+        tmin = fminf(tmin, fminf(fminf(out[0], out[1]), fminf(out[2], out[3])));
+        reinterpret_cast<float4*>(ncur)[mid] = make_float4(out[0], out[1], out[2], out[3]);
+        reinterpret_cast<float4*>(acur)[mid] = make_float4(aout[0], aout[1], aout[2], aout[3]);
+      }
+      tmin = -warp_max(-tmin);
+      if (lane == 0) wmin[(t & 1) * 32 + warp] = tmin;
+      if (tid == 0) hist_c[t] = C;
+      __syncthreads();
+      Rn = INFINITY;
+#pragma unroll
+      for (int w2 = 0; w2 < nwarps; ++w2) Rn = fminf(Rn, wmin[(t & 1) * 32 + w2]);
+    }
+    // log2 Z and Hbar = E[A_{n-1}]
     double l2Z;
-    float Hbar = 0.f;
+    float Hbar;
     {
-      const float* lfin = lb[(n - 1) & 1];
-      const float* afin = VJP ? hist_a + (size_t)(n - 1) * J : nullptr;
+      const float* nfin = lb[(n - 1) & 1];
+      const float* afin = bcg[(n - 1) & 1];
       float s0 = 0.f, s1 = 0.f;
       for (int j = tid; j < J; j += NT) {
-        const float u = ex2f(lfin[j] - R);
+        const float u = ex2f(Rn - nfin[j]);
         s0 += u;
-        if constexpr (VJP) s1 = fmaf(u, afin[j], s1);
+        s1 = fmaf(u, afin[j], s1);
       }
       s0 = warp_sum(s0);
-      if constexpr (VJP) s1 = warp_sum(s1);
+      s1 = warp_sum(s1);
       if (lane == 0) { part[warp * NP] = s0; part[warp * NP + 1] = s1; }
       __syncthreads();
       float a0 = 0.f, a1 = 0.f;
 #pragma unroll
       for (int w2 = 0; w2 < nwarps; ++w2) { a0 += part[w2 * NP]; a1 += part[w2 * NP + 1]; }
-      l2Z = (double)R + log2((double)a0) + C;
-      if constexpr (VJP) Hbar = a1 / a0;
-      if (MODE == MODE_SOFT && tid == 0 && P.out_logZ) P.out_logZ[seq] = (float)(l2Z * 0.69314718055994530942);
+      l2Z = -(double)Rn + log2((double)a0) + C;
+      Hbar = a1 / a0;
       __syncthreads();
     }
-    const float gzq = (VJP && P.gZ) ? P.gZ[seq] : 0.f;
-    const float hb = Hbar - gzq;
-    const float c2T = P.two_over_T / P.sk;
+    const float hb = Hbar - (P.gZ ? P.gZ[seq] : 0.f);
+    const float2 nc2T = f2s(-P.two_over_T / P.sk);
 
-    // ---------------------------------------------------------- backward
-    float Rr = 0.f;
-    double Cr = 0.0;
-    ld_cb(cs_tm, tid, cbn);
-    for (int t = n - 1; t >= 0; --t) {
-      const float* rcur = lb[t & 1];
-      float* rnext = lb[(t + 1) & 1];
-      const float* bcur = VJP ? bcg[t & 1] : nullptr;
-      float* bnext = VJP ? bcg[(t + 1) & 1] : nullptr;
-      const float wt = wsc[t];
-      const float gt = VJP ? gsc[t] : 0.f;
-      const float graw = gt * P.sk;
-      const double Csig = (t >= 1) ? hist_c[t - 1] : 0.0;
-      const float K = (float)(Csig + Cr - l2Z);
-      const bool last = (t == n - 1);
-      const float* hl = (t > 0) ? hist_l + (size_t)(t - 1) * J : nullptr;
-      const float* ha = (VJP && t > 0) ? hist_a + (size_t)(t - 1) * J : nullptr;
-      float acc0 = 0.f, acc1 = 0.f;  // SOFT: sum p c, sum p; VJP: sum G c, sum G
-      float bestp = -1.f;
-      int bestq = 0x7fffffff;
-      float tmax = -INFINITY;
-#pragma unroll
-      for (int k = 0; k < KB; ++k) {
-        const int mid = tid + NT * k;
-        float cb[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) cb[i] = cbn[i];
-        ld_cb(cs_tm, (k + 1 < KB) ? mid + NT : tid, cbn);
-        float r4[4], b4[4];
-        if (last) {
-#pragma unroll
-          for (int lo = 0; lo < 4; ++lo) { r4[lo] = 0.f; b4[lo] = 0.f; }
-        } else {
-          const float4 rv = reinterpret_cast<const float4*>(rcur)[mid];
-          r4[0] = rv.x; r4[1] = rv.y; r4[2] = rv.z; r4[3] = rv.w;
-          if constexpr (VJP) {
-            const float4 bv = reinterpret_cast<const float4*>(bcur)[mid];
-            b4[0] = bv.x; b4[1] = bv.y; b4[2] = bv.z; b4[3] = bv.w;
-          }
-        }
-        float gcb[16];
-        if constexpr (VJP) tmem_ld16(tbase + 16 * k, gcb);
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const int gi = (h << HB) | mid;
-          const float lsig = (t >= 1) ? hl[gi] : 0.f;
-          float asig = 0.f;
-          if constexpr (VJP) asig = (t >= 1) ? ha[gi] : 0.f;
-          float y[4], z[4];
-          float m = -INFINITY;
-#pragma unroll
-          for (int lo = 0; lo < 4; ++lo) {
-            const float d = wt - cb[4 * h + lo];
-            y[lo] = fmaf(-d, d, r4[lo]);
-            m = fmaxf(m, y[lo]);
-            if constexpr (VJP) z[lo] = fmaf(gt, cb[4 * h + lo], b4[lo]);
-          }
-          const float gf = ex2f(m + lsig + K);
-          float s = 0.f, num = 0.f;
-#pragma unroll
-          for (int lo = 0; lo < 4; ++lo) {
-            const float u = ex2f(y[lo] - m);
-            s += u;
-            const float p = u * gf;
-            if constexpr (MODE == MODE_SOFT) {
-              acc0 = fmaf(p, cb[4 * h + lo], acc0);
-              acc1 += p;
-              const int q = (h << 14) | (mid << 2) | lo;
-              arg_better(bestp, bestq, p, q);
-            } else {
-              num = fmaf(u, z[lo], num);
-              const float G = p * (asig + z[lo] - hb);
-              acc1 += G;
-              acc0 = fmaf(G, cb[4 * h + lo], acc0);
-              const float d = wt - cb[4 * h + lo];
-              gcb[4 * h + lo] = fmaf(c2T, G * d, fmaf(graw, p, gcb[4 * h + lo]));
-            }
-          }
-          if (t >= 1) {
-            const float l = m + lg2f(s) - Rr;
-            rnext[gi] = l;
-            tmax = fmaxf(tmax, l);
-            if constexpr (VJP) bnext[gi] = __fdividef(num, s);
-          }
-        }
-        if constexpr (VJP) tmem_st16(tbase + 16 * k, gcb);
-      }
-      if constexpr (VJP) tmem_wait_st();
-      acc0 = warp_sum(acc0);
-      acc1 = warp_sum(acc1);
-      tmax = warp_max(tmax);
-      if (MODE == MODE_SOFT) warp_argmax(bestp, bestq);
-      const int pb = t & 1;
-      if (lane == 0) {
-        part[(pb * 32 + warp) * NP] = acc0;
-        part[(pb * 32 + warp) * NP + 1] = acc1;
-        wmax[pb * 32 + warp] = tmax;
-        apart[pb * 32 + warp] = bestp;
-        aidx[pb * 32 + warp] = bestq;
-      }
-      __syncthreads();
-      if (tid == 0) {
-        float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-        for (int w2 = 0; w2 < nwarps; ++w2) { a0 += part[(pb * 32 + w2) * NP]; a1 += part[(pb * 32 + w2) * NP + 1]; }
-        if constexpr (MODE == MODE_SOFT) {
-          if (P.out_soft) P.out_soft[seq * P.len + t] = a0 / (a1 * P.sk);
-          if (P.out_argmax) {
-            float bp = -1.f;
-            int bq = 0x7fffffff;
-#pragma unroll
-            for (int w2 = 0; w2 < nwarps; ++w2) arg_better(bp, bq, apart[pb * 32 + w2], aidx[pb * 32 + w2]);
-            P.out_argmax[seq * n + t] = bq;
-          }
-        } else {
-          P.grad_w[seq * P.len + t] = P.two_over_T * (a0 / P.sk - (wt / P.sk) * a1);
-        }
-      }
-      Cr += (double)Rr;
-      Rr = -INFINITY;
-#pragma unroll
-      for (int w2 = 0; w2 < nwarps; ++w2) Rr = fmaxf(Rr, wmax[pb * 32 + w2]);
-    }
-
-    if constexpr (VJP) {
-      // fold this sequence's codebook gradient into the CTA partial and clear it
+    // tensor memory now accumulates this sequence's codebook gradient
+    {
       float z16[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) z16[i] = 0.f;
 #pragma unroll
+      for (int k = 0; k < KB; ++k) tmem_st16(tbase + 16 * k, z16);
+      tmem_wait_st();
+    }
+
+    // ------------------------------------------------------------ backward
+    // Work unit = one h-pair g of one block k: 8 states, 8 codewords, 8 TMEM
+    // columns; codewords and history values are prefetched one unit ahead.
+    float Rrn = 0.f;
+    double Cr = 0.0;
+    float cbn[8];
+    ld_cb8(cs_tm, tid, 0, cbn);
+    // block kk of step tt reads step tt-1's values (free start: 0 for tt = 0)
+    auto hist_at = [&](const float* hbuf, int tt, int kk) -> float4 {
+      return (tt >= 1) ? reinterpret_cast<const float4*>(hbuf + (size_t)(tt - 1) * J)[tid + NT * kk]
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    };
+    float4 hsn = hist_at(hist_l, n - 1, 0), han = hist_at(hist_a, n - 1, 0);
+    for (int t = n - 1; t >= 0; --t) {
+      const float* ncur = lb[t & 1];
+      float* nnext = lb[(t + 1) & 1];
+      const float* bcur = bcg[t & 1];
+      float* bnext = bcg[(t + 1) & 1];
+      const float nwt = wsc[t];
+      const float2 nw2 = f2s(nwt);
+      const float2 g2 = f2s(gsc[t]);
+      const float2 gr2 = f2s(gsc[t] * P.sk);
+      const double Csig = (t >= 1) ? hist_c[t - 1] : 0.0;
+      const float K = (float)(Csig + Cr - l2Z);
+      const bool last = (t == n - 1);
+      float2 accG = f2s(0.f), accGc = f2s(0.f);
+      float tmin = INFINITY;
+      float4 bvn = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (!last) bvn = reinterpret_cast<const float4*>(bcur)[tid];
+#pragma unroll
       for (int k = 0; k < KB; ++k) {
         const int mid = tid + NT * k;
-        float gcb[16];
-        tmem_ld16(tbase + 16 * k, gcb);
-        double* dst = gcp + (size_t)mid * 16;
+        float nr[4], bc[4];
+        if (last) {
+          nr[0] = nr[1] = nr[2] = nr[3] = 0.f;
+          bc[0] = bc[1] = bc[2] = bc[3] = 0.f;
+        } else {
+          const float4 rv = reinterpret_cast<const float4*>(ncur)[mid];
+          nr[0] = rv.x; nr[1] = rv.y; nr[2] = rv.z; nr[3] = rv.w;
+          bc[0] = bvn.x; bc[1] = bvn.y; bc[2] = bvn.z; bc[3] = bvn.w;
+        }
+        if (!last && k + 1 < KB) bvn = reinterpret_cast<const float4*>(bcur)[mid + NT];
+        const float4 hs4 = hsn, ha4 = han;
+        {
+          const int nt = (k + 1 < KB) ? t : t - 1, nk = (k + 1 < KB) ? k + 1 : 0;
+          hsn = hist_at(hist_l, nt, nk);
+          han = hist_at(hist_a, nt, nk);
+        }
+        float nout[4], bout[4];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) dst[i] += (double)gcb[i];
-        tmem_st16(tbase + 16 * k, z16);
+        for (int g = 0; g < 2; ++g) {          // groups h = 2g, 2g+1 side by side
+          float cb[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) cb[i] = cbn[i];
+          const float hs0 = g ? hs4.z : hs4.x, hs1 = g ? hs4.w : hs4.y;
+          const float ha0 = g ? ha4.z : ha4.x, ha1 = g ? ha4.w : ha4.y;
+          {
+            // codewords of the unit after (k, g): (k, 1), (k+1, 0) or (0, 0)
+            const int nk = (g == 0) ? k : ((k + 1 < KB) ? k + 1 : 0);
+            ld_cb8(cs_tm, tid + NT * nk, (g == 0) ? 1 : 0, cbn);
+          }
+          float gcb[8];
+          tmem_ld8(tbase + 16 * k + 8 * g, gcb);
+          float2 y[4], c2[4], d2[4];
+#pragma unroll
+          for (int lo = 0; lo < 4; ++lo) {
+            c2[lo] = f2(cb[2 * lo], cb[2 * lo + 1]);
+            d2[lo] = __fadd2_rn(c2[lo], nw2);
+            y[lo] = __ffma2_rn(d2[lo], d2[lo], f2s(nr[lo]));
+          }
+          const float2 m = f2(fminf(fminf(y[0].x, y[1].x), fminf(y[2].x, y[3].x)),
+                              fminf(fminf(y[0].y, y[1].y), fminf(y[2].y, y[3].y)));
+          const float2 ge = __fadd2_rn(__fadd2_rn(f2s(K), f2(-hs0, -hs1)), __fmul2_rn(m, neg1));
+          const float2 gf = f2(ex2f(ge.x), ex2f(ge.y));
+          const float2 ah = f2(ha0 - hb, ha1 - hb);   // A - Hbar + gZ
+          float2 ssum = f2s(0.f), num = f2s(0.f);
+#pragma unroll
+          for (int lo = 0; lo < 4; ++lo) {
+            const float2 a = __ffma2_rn(y[lo], neg1, m);
+            const float2 u = f2(ex2f(a.x), ex2f(a.y));
+            ssum = __fadd2_rn(ssum, u);
+            const float2 z = __ffma2_rn(g2, c2[lo], f2s(bc[lo]));          // Bc + h
+            num = __ffma2_rn(u, z, num);
+            const float2 pp = __fmul2_rn(u, gf);
+            const float2 G = __fmul2_rn(pp, __fadd2_rn(z, ah));
+            accG = __fadd2_rn(accG, G);
+            accGc = __ffma2_rn(G, c2[lo], accGc);
+            float2 gc = f2(gcb[2 * lo], gcb[2 * lo + 1]);
+            gc = __ffma2_rn(gr2, pp, gc);
+            gc = __ffma2_rn(__fmul2_rn(G, d2[lo]), nc2T, gc);              // + (2/T) G (w - c)
+            gcb[2 * lo] = gc.x;
+            gcb[2 * lo + 1] = gc.y;
+          }
+          tmem_st8(tbase + 16 * k + 8 * g, gcb);
+          nout[2 * g] = (m.x - Rrn) - lg2f(ssum.x);
+          nout[2 * g + 1] = (m.y - Rrn) - lg2f(ssum.y);
+          bout[2 * g] = __fdividef(num.x, ssum.x);
+          bout[2 * g + 1] = __fdividef(num.y, ssum.y);
+        }
+        if (t >= 1) {
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            nnext[(h << HB) | mid] = nout[h];
+            bnext[(h << HB) | mid] = bout[h];
+          }
+          tmin = fminf(tmin, fminf(fminf(nout[0], nout[1]), fminf(nout[2], nout[3])));
+        }
       }
       tmem_wait_st();
+      const float a0 = warp_sum(accGc.x + accGc.y);
+      const float a1 = warp_sum(accG.x + accG.y);
+      tmin = -warp_max(-tmin);
+      const int pb = t & 1;
+      if (lane == 0) {
+        part[(pb * 32 + warp) * NP] = a0;
+        part[(pb * 32 + warp) * NP + 1] = a1;
+        wmin[pb * 32 + warp] = tmin;
+      }
+      __syncthreads();
+      if (tid == 0) {
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int w2 = 0; w2 < nwarps; ++w2) { s0 += part[(pb * 32 + w2) * NP]; s1 += part[(pb * 32 + w2) * NP + 1]; }
+        // dl/dw_t = (2/T) (sum G c - w_t sum G), c = c'/sk, w_t = -nwt/sk
+        P.grad_w[seq * P.len + t] = P.two_over_T * (s0 + nwt * s1) / P.sk;
+      }
+      Cr -= (double)Rrn;
+      Rrn = INFINITY;
+#pragma unroll
+      for (int w2 = 0; w2 < nwarps; ++w2) Rrn = fminf(Rrn, wmin[pb * 32 + w2]);
+    }
+
+    // fold this sequence's codebook gradient into the CTA partial
+#pragma unroll
+    for (int k = 0; k < KB; ++k) {
+      const int mid = tid + NT * k;
+      float gcb[16];
+      tmem_ld16(tbase + 16 * k, gcb);
+      double* dst = gcp + (size_t)mid * 16;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) dst[i] += (double)gcb[i];
     }
     __syncthreads();
   }
 
-  if constexpr (VJP) {
-    tmem_fence_before();
-    __syncthreads();
-    tmem_fence_after();
-    if (warp == 0) tmem_dealloc512(tslot[0]);
-  }
+  tmem_fence_before();
+  __syncthreads();
+  tmem_fence_after();
+  if (warp == 0) tmem_dealloc512(tslot[0]);
 }
 
 }  // namespace l16

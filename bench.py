@@ -314,6 +314,7 @@ def main():
                        "parallelism": f"dp{world}" if world > 1 else "single"},
             "weights_per_s": world * wl.n_seq * wl.seq_len / (ms_step / 1e3),
             "ms_soft": ms_soft, "ms_vjp": ms_vjp, "wall_s": wall,
+            "ms_step_min_max": [min(step_ms), max(step_ms)],
             "gpu_launches": 5 * args.steps,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks}
     print(json.dumps(line), flush=True)

@@ -31,9 +31,12 @@
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
  *     stream).  Calls are asynchronous: they validate their arguments, enqueue
  *     the work on `stream` and return.  Argument errors are returned at once and
- *     enqueue nothing.  The library allocates its own scratch space with
- *     cudaMallocAsync on `stream` and frees it on `stream` before returning;
- *     it keeps no state between calls.
+ *     enqueue nothing.  The library allocates its own scratch space, stream-
+ *     ordered on `stream`, from a library-private memory pool of the current
+ *     device and frees it on `stream` before returning; freed scratch stays
+ *     mapped in that pool for reuse by later calls (up to the largest call's
+ *     size, several GB for L=16, until the process exits).  No data is kept
+ *     between calls.
  *   - Supported: 1 <= D = k*V <= L <= 16, D <= 6, V in {1, 2, 4},
  *     len <= 8192; T finite and > 0.  n_seq == 0 is a no-op returning BCJR_OK.
  *   - Errors: null or non-device pointers, len not a positive multiple of V,
