@@ -540,8 +540,9 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
     // columns; codewords and history values are prefetched one unit ahead.
     float Rrn = 0.f;
     double Cr = 0.0;
-    float cbn[8];
+    float cbn[8], cbm[8];
     ld_cb8(cs_tm, tid, 0, cbn);
+    ld_cb8(cs_tm, tid, 1, cbm);
     // block kk of step tt reads step tt-1's values (free start: 0 for tt = 0)
     auto hist_at = [&](const float* hbuf, int tt, int kk) -> float4 {
       return (tt >= 1) ? reinterpret_cast<const float4*>(hbuf + (size_t)(tt - 1) * J)[tid + NT * kk]
@@ -588,22 +589,22 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
         for (int g = 0; g < 2; ++g) {          // groups h = 2g, 2g+1 side by side
           float cb[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) cb[i] = cbn[i];
+          for (int i = 0; i < 8; ++i) { cb[i] = cbn[i]; cbn[i] = cbm[i]; }
           const float hs0 = g ? hs4.z : hs4.x, hs1 = g ? hs4.w : hs4.y;
           const float ha0 = g ? ha4.z : ha4.x, ha1 = g ? ha4.w : ha4.y;
           {
-            // codewords of the unit after (k, g): (k, 1), (k+1, 0) or (0, 0)
-            const int nk = (g == 0) ? k : ((k + 1 < KB) ? k + 1 : 0);
-            ld_cb8(cs_tm, tid + NT * nk, (g == 0) ? 1 : 0, cbn);
+            // codewords two units after (k, g): block k+1 (or 0), same g
+            const int nk = (k + 1 < KB) ? k + 1 : 0;
+            ld_cb8(cs_tm, tid + NT * nk, g, cbm);
           }
           float gcb[8];
           tmem_ld8(tbase + 16 * k + 8 * g, gcb);
-          float2 y[4], c2[4], d2[4];
+          float2 y[4], c2[4];
 #pragma unroll
           for (int lo = 0; lo < 4; ++lo) {
             c2[lo] = f2(cb[2 * lo], cb[2 * lo + 1]);
-            d2[lo] = __fadd2_rn(c2[lo], nw2);
-            y[lo] = __ffma2_rn(d2[lo], d2[lo], f2s(nr[lo]));
+            const float2 dd = __fadd2_rn(c2[lo], nw2);
+            y[lo] = __ffma2_rn(dd, dd, f2s(nr[lo]));
           }
           const float2 m = f2(fminf(fminf(y[0].x, y[1].x), fminf(y[2].x, y[3].x)),
                               fminf(fminf(y[0].y, y[1].y), fminf(y[2].y, y[3].y)));
@@ -624,7 +625,7 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
             accGc = __ffma2_rn(G, c2[lo], accGc);
             float2 gc = f2(gcb[2 * lo], gcb[2 * lo + 1]);
             gc = __ffma2_rn(gr2, pp, gc);
-            gc = __ffma2_rn(__fmul2_rn(G, d2[lo]), nc2T, gc);              // + (2/T) G (w - c)
+            gc = __ffma2_rn(__fmul2_rn(G, __fadd2_rn(c2[lo], nw2)), nc2T, gc);  // + (2/T) G (w - c)
             gcb[2 * lo] = gc.x;
             gcb[2 * lo + 1] = gc.y;
           }
