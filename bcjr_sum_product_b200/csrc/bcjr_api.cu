@@ -99,6 +99,13 @@ int check_shape(int64_t n_seq, int64_t len, int L, int k, int V, Shape* sh) {
   return BCJR_OK;
 }
 
+// BCJR_GENERIC_ONLY=1 routes every call to the generic kernels (used by tests
+// that compare the specialised kernels against them).
+bool generic_only() {
+  const char* e = std::getenv("BCJR_GENERIC_ONLY");
+  return e && e[0] == '1';
+}
+
 int check_T(float T) { return (std::isfinite(T) && T > 0.f) ? BCJR_OK : BCJR_ERR_INVALID_ARG; }
 
 // Carves one stream-ordered allocation into 256-byte aligned pieces.
@@ -203,11 +210,7 @@ int run_l16(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   return BCJR_OK;
 }
 
-bool use_l16(const Shape& sh) {
-  const char* e = std::getenv("BCJR_GENERIC_ONLY");
-  if (e && e[0] == '1') return false;
-  return sh.L == 16 && sh.D == 2 && sh.V == 1;
-}
+bool use_l16(const Shape& sh) { return !generic_only() && sh.L == 16 && sh.D == 2 && sh.V == 1; }
 
 template <int MODE>
 int run_sweep(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
@@ -274,8 +277,45 @@ ViterbiKernel pick_viterbi(int V, int D) {
   return nullptr;
 }
 
+// L = 16, D = 2, V = 1: the block-layout Viterbi of bcjr_l16.cuh.
+int run_viterbi_l16(const Shape& sh, const float* w, const float* c, int32_t* out_states, float* out_cost,
+                    cudaStream_t st) {
+  namespace K = bcjr::l16;
+  const size_t smem = sizeof(float) * ((size_t)2 * K::J + 32 + 32 + 64 + 4 + (size_t)sh.n);
+  if (smem > kMaxDynSmem) return BCJR_ERR_UNSUPPORTED;
+  int grid = 0;
+  int rc = grid_for(K::viterbi_kernel, K::NT, smem, sh.n_seq, &grid);
+  if (rc != BCJR_OK) return rc;
+  // backpointer batch per CTA: up to 16 sequences, within about 2.5 GB in total
+  const size_t per_seq = (size_t)sh.n * K::NMID;
+  int64_t tb = (int64_t)(2500000000ull / ((size_t)grid * per_seq));
+  if (tb > 16) tb = 16;
+  if (tb < 1) tb = 1;
+  K::VParams P{};
+  auto layout = [&](Arena& ar) {
+    P.cb_raw = ar.take<float>(K::S);
+    P.bp = ar.take<uint8_t>((size_t)grid * tb * per_seq);
+  };
+  Arena sizing;
+  layout(sizing);
+  void* mem = nullptr;
+  if (int arc = scratch_alloc(&mem, sizing.off, st)) return arc;
+  Arena ar;
+  ar.base = static_cast<char*>(mem);
+  layout(ar);
+  P.w = w; P.out_states = out_states; P.out_cost = out_cost;
+  P.n_seq = sh.n_seq; P.len = sh.len; P.n = sh.n; P.tb = (int)tb;
+  K::make_block_codebook<<<K::S / 256, 256, 0, st>>>(c, 1.0f, const_cast<float*>(P.cb_raw));
+  K::viterbi_kernel<<<grid, K::NT, smem, st>>>(P);
+  cudaError_t le = cudaGetLastError();
+  cudaError_t fe = cudaFreeAsync(mem, st);
+  if (le != cudaSuccess || fe != cudaSuccess) return BCJR_ERR_CUDA;
+  return BCJR_OK;
+}
+
 int run_viterbi(const Shape& sh, const float* w, const float* c, int32_t* out_states, float* out_cost,
                 cudaStream_t st) {
+  if (sh.L == 16 && sh.D == 2 && sh.V == 1 && !generic_only()) return run_viterbi_l16(sh, w, c, out_states, out_cost, st);
   ViterbiKernel kern = pick_viterbi(sh.V, sh.D);
   if (!kern) return BCJR_ERR_UNSUPPORTED;
   const int threads = threads_for(sh.J);

@@ -687,5 +687,162 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
   if (warp == 0) tmem_dealloc512(tslot[0]);
 }
 
+
+// ------------------------------------------------------------ Viterbi
+// The T -> 0 decode in the same block layout: per step and forward group
+// j = (mid << 2) | lo, mu_t(j) = min_h delta_t((h << 14) | j) with
+// delta_t(q) = fl(mu_{t-1}(q >> 2) + fl(fl(w_t - c(q))^2)) (delta_0 = q_0),
+// the lowest h winning ties.  The four 2-bit backpointers of a block form one
+// byte per step.  A CTA decodes a batch of up to TB sequences, then traces
+// them back in parallel (one thread per sequence).  The arithmetic is the
+// prescribed fp32 sequence in scalar IEEE round-to-nearest operations that
+// are never fused (the packed f32x2 forms gave 1-ulp differences in the
+// accumulated cost on this hardware, so they are not used here).
+struct VParams {
+  const float* w;       // [n_seq][len]
+  const float* cb_raw;  // block-major raw codebook [4096][16]
+  int32_t* out_states;  // [n_seq][n]
+  float* out_cost;      // [n_seq] or null
+  uint8_t* bp;          // [grid][TB][n][NMID]
+  int64_t n_seq, len;
+  int n, tb;
+};
+
+__global__ void __launch_bounds__(NT, 1) viterbi_kernel(VParams P) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int nwarps = NT / 32;
+  const int n = P.n, TB = P.tb;
+  extern __shared__ __align__(16) float smem[];
+  float* mb[2] = {smem, smem + J};
+  float* redv = smem + 2 * J;                          // [32]
+  int* redq = reinterpret_cast<int*>(redv + 32);       // [32]
+  int* fin = redq + 32;                                // [TB] final state per sequence of the batch
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(fin + 64);  // [4]
+  float* wsm = reinterpret_cast<float*>(tslot + 4);    // n: w
+  uint8_t* bp = P.bp + (size_t)blockIdx.x * TB * n * NMID;
+
+  if (warp == 0) tmem_alloc512(tslot);
+  tmem_fence_before();
+  __syncthreads();
+  tmem_fence_after();
+  const uint32_t tbase = tslot[0] + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(128 * (warp >> 2));
+#pragma unroll
+  for (int k = 0; k < KB; ++k) {
+    float c16[16];
+    ld_cb(P.cb_raw, tid + NT * k, c16);
+    tmem_st16(tbase + 16 * k, c16);
+  }
+  tmem_wait_st();
+
+  const int64_t stride = (int64_t)gridDim.x;
+  for (int64_t base = blockIdx.x; base < P.n_seq; base += stride * TB) {
+    int nb = 0;
+    for (int i = 0; i < TB; ++i, ++nb) {
+      const int64_t seq = base + i * stride;
+      if (seq >= P.n_seq) break;
+      const float* wq = P.w + seq * P.len;
+      for (int x = tid; x < n; x += NT) wsm[x] = wq[x];
+      __syncthreads();
+      uint8_t* bpi = bp + (size_t)i * n * NMID;
+      float bestv = INFINITY;
+      int bestq = 0x7fffffff;
+      for (int t = 0; t < n; ++t) {
+        const float* mprev = mb[(t + 1) & 1];
+        float* mcur = mb[t & 1];
+        const float wv = wsm[t];
+        const bool last = (t == n - 1);
+#pragma unroll
+        for (int k = 0; k < KB; ++k) {
+          const int mid = tid + NT * k;
+          float cb[16];
+          tmem_ld16(tbase + 16 * k, cb);
+          float2 mp01 = f2s(0.f), mp23 = f2s(0.f);
+          if (t > 0) {
+            mp01 = f2(mprev[(0 << HB) | mid], mprev[(1 << HB) | mid]);
+            mp23 = f2(mprev[(2 << HB) | mid], mprev[(3 << HB) | mid]);
+          }
+          float mout[4];
+          uint32_t byte = 0;
+#pragma unroll
+          for (int lo = 0; lo < 4; ++lo) {
+            // scalar IEEE operations in the prescribed order: q = fl(fl(w - c)^2), delta = fl(mu + q)
+            float e[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const float d = __fsub_rn(wv, cb[bidx(h, lo)]);
+              e[h] = __fmul_rn(d, d);
+            }
+            if (t > 0) {
+              e[0] = __fadd_rn(mp01.x, e[0]); e[1] = __fadd_rn(mp01.y, e[1]);
+              e[2] = __fadd_rn(mp23.x, e[2]); e[3] = __fadd_rn(mp23.y, e[3]);
+            }
+            const float2 e01 = f2(e[0], e[1]), e23 = f2(e[2], e[3]);
+            float b = e01.x;
+            uint32_t bh = 0;
+            if (e01.y < b) { b = e01.y; bh = 1; }
+            if (e23.x < b) { b = e23.x; bh = 2; }
+            if (e23.y < b) { b = e23.y; bh = 3; }
+            mout[lo] = b;
+            byte |= bh << (2 * lo);
+            if (last) {
+              const float dv[4] = {e01.x, e01.y, e23.x, e23.y};
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const int q = (h << 14) | (mid << 2) | lo;
+                if (dv[h] < bestv || (dv[h] == bestv && q < bestq)) { bestv = dv[h]; bestq = q; }
+              }
+            }
+          }
+          reinterpret_cast<float4*>(mcur)[mid] = make_float4(mout[0], mout[1], mout[2], mout[3]);
+          if (!last) bpi[(size_t)t * NMID + mid] = (uint8_t)byte;
+        }
+        __syncthreads();
+      }
+      // argmin of delta_{n-1} over all states, lowest state on ties
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float v2 = __shfl_xor_sync(0xffffffffu, bestv, o);
+        const int q2 = __shfl_xor_sync(0xffffffffu, bestq, o);
+        if (v2 < bestv || (v2 == bestv && q2 < bestq)) { bestv = v2; bestq = q2; }
+      }
+      if (lane == 0) { redv[warp] = bestv; redq[warp] = bestq; }
+      __syncthreads();
+      if (tid == 0) {
+        float bv = INFINITY;
+        int bq = 0x7fffffff;
+#pragma unroll
+        for (int w2 = 0; w2 < nwarps; ++w2)
+          if (redv[w2] < bv || (redv[w2] == bv && redq[w2] < bq)) { bv = redv[w2]; bq = redq[w2]; }
+        if (bq == 0x7fffffff) bq = 0;  // all-NaN sequence
+        fin[i] = bq;
+        if (P.out_cost) P.out_cost[seq] = bv;
+      }
+      __syncthreads();
+    }
+    // trace the batch back, one thread per sequence
+    if (tid < nb) {
+      const int i = tid;
+      const int64_t seq = base + i * stride;
+      const uint8_t* bpi = bp + (size_t)i * n * NMID;
+      int32_t* out = P.out_states + seq * n;
+      int st = fin[i];
+      for (int t = n - 1; t >= 0; --t) {
+        out[t] = st;
+        if (t > 0) {
+          const int jp = st >> 2;   // group of the predecessors at step t-1
+          const int h = (bpi[(size_t)(t - 1) * NMID + (jp >> 2)] >> (2 * (jp & 3))) & 3;
+          st = jp | (h << 14);
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  tmem_fence_before();
+  __syncthreads();
+  tmem_fence_after();
+  if (warp == 0) tmem_dealloc512(tslot[0]);
+}
+
 }  // namespace l16
 }  // namespace bcjr

@@ -173,3 +173,20 @@ def test_l16_block_kernel_matches_generic_kernel(monkeypatch):
     assert_soft(fast[0][rows], ref["soft"], c)
     rv = oracle.vjp(w[rows], c, 16, 2, 1, 0.05, g[rows], gZ[rows])
     assert_grad(fast[2][rows], rv["grad_w"], "grad_w")
+
+
+def test_l16_viterbi_matches_generic_and_oracle(monkeypatch):
+    """The block-layout L=16 Viterbi against the generic kernel (bit-exact) on
+    40 sequences of 96 steps, including exact ties from a coarse codebook."""
+    w, c, _ = I.random_case(16, 2, 1, 40, 96, seed=515)
+    c[::7] = torch.round(c[::7] * 4) / 4
+    w[:5] = torch.round(w[:5] * 4) / 4
+    wd, cd = w.to(DEV), c.to(DEV)
+    s_fast, c_fast = lib.viterbi_decode(wd, cd, 16, 2, 1)
+    monkeypatch.setenv("BCJR_GENERIC_ONLY", "1")
+    s_gen, c_gen = lib.viterbi_decode(wd, cd, 16, 2, 1)
+    torch.cuda.synchronize()
+    assert torch.equal(s_fast, s_gen) and torch.equal(c_fast, c_gen)
+    ref = oracle.viterbi(w[:6], c, 16, 2, 1)
+    np.testing.assert_array_equal(s_fast[:6].cpu().numpy(), ref["states"])
+    np.testing.assert_array_equal(c_fast[:6].cpu().numpy(), ref["cost"])
