@@ -42,6 +42,10 @@ LEDGER = {
     "soft": {"fp32": 3.75 + 6.75, "mufu": 2.0},
     "vjp": {"fp32": 7.5 + 16.5, "mufu": 2.0},
 }
+# DRAM bytes per sequence (read + write) of each L=16 sweep kernel, from one
+# ncu capture of 16 qtip sequences (profiles/vjp_kernel_qtip16.md,
+# profiles/soft_kernel_qtip16.md); set to None whenever the kernel changes.
+TRAFFIC_PER_SEQ = {"vjp": 1000.66e6 / 16, "soft": 443.68e6 / 16}
 FP32_PER_CLK_SM = 128.0   # FFMA lanes per SM per clock (measured 123.5 FFMA, 126 FFMA2 on this machine)
 MUFU_PER_CLK_SM = 16.0    # ex2 per SM per clock (measured 15.99 on this machine)
 N_SM = 148
@@ -172,12 +176,15 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--seqs", type=int, default=0,
+                    help="profiling only: run on the first N sequences of the workload (not a bench number)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
 
     import torch
     import torch.distributed as dist
+    from bcjr_sum_product_b200 import dist as bdist
     from bcjr_sum_product_b200 import inputs as I
     from bcjr_sum_product_b200 import lib
 
@@ -193,20 +200,23 @@ def main():
     lib.load()
 
     wl = I.WORKLOADS[WORKLOAD]
-    inp = I.make(WORKLOAD)
+    inp = I.make(WORKLOAD, rows=list(range(args.seqs)) if args.seqs > 0 else None)
     T = wl.temps[0]
     L, k, V = wl.L, wl.k, wl.V
+    n_seq = inp.w.shape[0]
     stream = torch.cuda.current_stream(dev)
     w = inp.w.to(dev); c = inp.c.to(dev); g = inp.g.to(dev)
-    soft = torch.empty_like(w); logZ = torch.empty(wl.n_seq, device=dev)
+    soft = torch.empty_like(w); logZ = torch.empty(n_seq, device=dev)
     gw = torch.empty_like(w); gc = torch.empty_like(c)
     flush = torch.empty(256 * 1024 * 1024 // 4, device=dev)  # 256 MB > 126 MB L2
 
+    def local_vjp(wl_, cb_, g_):
+        return lib.vjp(wl_, cb_, L, k, V, T, g_, grad_w=gw, grad_codebook=gc, stream=stream)
+
     def step():
         lib.soft_codeword(w, c, L, k, V, T, out_soft=soft, out_logZ=logZ, stream=stream)
-        lib.vjp(w, c, L, k, V, T, g, grad_w=gw, grad_codebook=gc, stream=stream)
-        if world > 1:
-            dist.all_reduce(gc)
+        # each rank: VJP of its own sequences, then the codebook gradient summed over ranks
+        bdist.vjp_data_parallel(local_vjp, w, c, g)
 
     for _ in range(args.warmup):
         step()
@@ -227,9 +237,7 @@ def main():
         e0.record(stream)
         lib.soft_codeword(w, c, L, k, V, T, out_soft=soft, out_logZ=logZ, stream=stream)
         e1.record(stream)
-        lib.vjp(w, c, L, k, V, T, g, grad_w=gw, grad_codebook=gc, stream=stream)
-        if world > 1:
-            dist.all_reduce(gc)
+        bdist.vjp_data_parallel(local_vjp, w, c, g)
         e2.record(stream)
         e2.synchronize()
         soft_ms.append(e0.elapsed_time(e1)); vjp_ms.append(e1.elapsed_time(e2)); step_ms.append(e0.elapsed_time(e2))
@@ -246,14 +254,14 @@ def main():
     ms_step = float(total[0]) / args.steps
     ms_soft = float(total[1]) / args.steps
     ms_vjp = float(total[2]) / args.steps
-    units = wl.units
+    units = n_seq * wl.n_steps * wl.S
     value = world * units / (ms_step / 1e3)
 
     # e2e: through the public API with host buffers, copies inside the timed region
     e2e = None
     if not args.no_e2e:
         hw = inp.w.pin_memory(); hc = inp.c.pin_memory(); hg = inp.g.pin_memory()
-        out_soft_h = torch.empty_like(hw).pin_memory(); out_logZ_h = torch.empty(wl.n_seq).pin_memory()
+        out_soft_h = torch.empty_like(hw).pin_memory(); out_logZ_h = torch.empty(n_seq).pin_memory()
         out_gw_h = torch.empty_like(hw).pin_memory(); out_gc_h = torch.empty_like(hc).pin_memory()
         h2d = hw.numel() * 4 + hc.numel() * 4 + hg.numel() * 4
         d2h = out_soft_h.numel() * 4 + out_logZ_h.numel() * 4 + out_gw_h.numel() * 4 + out_gc_h.numel() * 4
@@ -265,9 +273,7 @@ def main():
             a.record(stream)
             w.copy_(hw, non_blocking=True); c.copy_(hc, non_blocking=True); g.copy_(hg, non_blocking=True)
             lib.soft_codeword(w, c, L, k, V, T, out_soft=soft, out_logZ=logZ, stream=stream)
-            lib.vjp(w, c, L, k, V, T, g, grad_w=gw, grad_codebook=gc, stream=stream)
-            if world > 1:
-                dist.all_reduce(gc)
+            bdist.vjp_data_parallel(local_vjp, w, c, g)
             out_soft_h.copy_(soft, non_blocking=True); out_logZ_h.copy_(logZ, non_blocking=True)
             out_gw_h.copy_(gw, non_blocking=True); out_gc_h.copy_(gc, non_blocking=True)
             b.record(stream)
@@ -291,8 +297,10 @@ def main():
     ms_dom = ms_vjp if dominant == "vjp" else ms_soft
     achieved = units / (ms_dom / 1e3)
     peak = peak_units_per_s(dominant, fmax)
-    roofline = {"bound": "alu", "kernel": f"bcjr_sweep_kernel ({dominant})", "achieved": achieved, "peak": peak,
-                "unit": UNIT, "frac": achieved / peak, "traffic": None,
+    tps = TRAFFIC_PER_SEQ.get(dominant)
+    roofline = {"bound": "alu", "kernel": f"bcjr::l16::{dominant}_kernel", "achieved": achieved, "peak": peak,
+                "unit": UNIT, "frac": achieved / peak, "traffic": (tps * n_seq) if tps else None,
+                "traffic_note": "DRAM bytes per launch, scaled from an ncu capture of 16 sequences",
                 "peak_basis": f"{N_SM} SMs x min(128 FP32 / {LEDGER[dominant]['fp32']}, 16 MUFU / "
                               f"{LEDGER[dominant]['mufu']}) units/clk at sm_max {fmax:.0f} MHz ({basis})",
                 "step_frac": value / world / peak_units_per_s("step", fmax)}
@@ -300,23 +308,29 @@ def main():
         roofline["frac_at_sampled_clock"] = achieved / peak_units_per_s(dominant, clocks["sm_mhz"])
 
     cpu = None
+    if args.seqs > 0:
+        line_note = f"profiling subset: first {n_seq} sequences only, not a bench number"
+    else:
+        line_note = None
     if world == 1 and not args.no_cpu_baseline:
         cores = os.cpu_count() or 1
-        cpu = cpu_baseline(wl, inp, max(1, min(cores, 16)))
+        cpu = cpu_baseline(wl, inp, max(1, min(cores, 16, n_seq)))
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": f"{wl.name}: L=16 k=2 V=1, 2048x2048 fp32 matrix as {wl.n_seq} x 256-weight "
                                    f"sequences, T=0.05, soft codeword + logZ + VJP per step",
-                       "n_seq_per_gpu": wl.n_seq, "steps_per_seq": wl.n_steps, "states": wl.S,
+                       "n_seq_per_gpu": n_seq, "steps_per_seq": wl.n_steps, "states": wl.S,
                        "l2": "flushed between timed iterations (256 MB write outside the events)",
                        "parallelism": f"dp{world}" if world > 1 else "single"},
-            "weights_per_s": world * wl.n_seq * wl.seq_len / (ms_step / 1e3),
+            "weights_per_s": world * n_seq * wl.seq_len / (ms_step / 1e3),
             "ms_soft": ms_soft, "ms_vjp": ms_vjp, "wall_s": wall,
             "ms_step_min_max": [min(step_ms), max(step_ms)],
             "gpu_launches": 5 * args.steps,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks}
+    if line_note:
+        line["note"] = line_note
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
