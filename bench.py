@@ -45,7 +45,7 @@ LEDGER = {
 # DRAM bytes per sequence (read + write) of each L=16 sweep kernel, from one
 # ncu capture of 16 qtip sequences (profiles/vjp_kernel_qtip16.md,
 # profiles/soft_kernel_qtip16.md); set to None whenever the kernel changes.
-TRAFFIC_PER_SEQ = {"vjp": 1000.66e6 / 16, "soft": 443.68e6 / 16}
+TRAFFIC_PER_SEQ = {"vjp": 1002.29e6 / 16, "soft": 445.70e6 / 16}
 FP32_PER_CLK_SM = 128.0   # FFMA lanes per SM per clock (measured 123.5 FFMA, 126 FFMA2 on this machine)
 MUFU_PER_CLK_SM = 16.0    # ex2 per SM per clock (measured 15.99 on this machine)
 N_SM = 148
