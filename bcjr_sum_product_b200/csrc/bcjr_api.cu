@@ -141,6 +141,23 @@ int grid_for(K kernel, int threads, size_t smem, int64_t n_seq, int* grid) {
   return BCJR_OK;
 }
 
+// Fewer resident CTAs when their per-CTA scratch (histories grow with the
+// sequence length) would exceed half of the free device memory or 24 GiB.
+void cap_grid_by_memory(int* grid, size_t per_cta_bytes) {
+  size_t free_b = 0, total_b = 0;
+  if (cudaMemGetInfo(&free_b, &total_b) != cudaSuccess) {
+    cudaGetLastError();
+    return;
+  }
+  size_t budget = free_b / 2;
+  const size_t cap = (size_t)24 << 30;
+  if (budget > cap) budget = cap;
+  if (per_cta_bytes == 0) return;
+  size_t g = budget / per_cta_bytes;
+  if (g < 1) g = 1;
+  if ((size_t)*grid > g) *grid = (int)g;
+}
+
 // ----------------------------------------------------------------- sweep
 using SweepKernel = void (*)(SweepParams);
 
@@ -175,11 +192,15 @@ int run_l16(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   constexpr bool VJP = MODE == bcjr::MODE_VJP;
   void (*kern)(K::Params) = K::vjp_kernel;
   if (!VJP) kern = a.out_argmax ? K::soft_kernel<true> : K::soft_kernel<false>;
-  const size_t smem = sizeof(float) * ((size_t)2 * K::J + 64 + 2 * 32 * 2 + 64 + 64 + 4 + 2 * (size_t)sh.n);
+  // state ping-pong, per-warp partials, TMEM slot, per-step weights (and gradients)
+  const size_t smem = sizeof(float) * ((size_t)2 * K::J + (VJP ? 2 * 32 * 8 : 64 + 2 * 32 * 2 + 64 + 64) + 4 +
+                                       (VJP ? 2 : 1) * (size_t)sh.n);
   if (smem > kMaxDynSmem) return BCJR_ERR_UNSUPPORTED;
   int grid = 0;
   int rc = grid_for(kern, K::NT, smem, sh.n_seq, &grid);
   if (rc != BCJR_OK) return rc;
+  cap_grid_by_memory(&grid, sizeof(float) * (size_t)sh.n * K::J * (VJP ? 2 : 1) + sizeof(double) * sh.n +
+                                (VJP ? sizeof(float) * 2 * K::J + sizeof(double) * K::S : 0));
   K::Params P{};
   auto layout = [&](Arena& ar) {
     P.cs_tm = ar.take<float>(K::S);
@@ -219,8 +240,8 @@ int run_sweep(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   SweepKernel kern = pick_sweep<MODE>(sh.V, sh.D);
   if (!kern) return BCJR_ERR_UNSUPPORTED;
   const int threads = threads_for(sh.J);
-  const int NP = sh.V + 1;
-  size_t fixed = sizeof(float) * ((size_t)sh.n * sh.V * (VJP ? 2 : 1) + 64 + 64 * NP + 64 + 64);
+  const int NPT = sh.V + 1 + (VJP ? 3 : 0);   // per-warp partials per step
+  size_t fixed = sizeof(float) * ((size_t)sh.n * sh.V * (VJP ? 2 : 1) + 64 + 64 * NPT + 64 + 64);
   size_t state_bytes = sizeof(float) * (size_t)sh.J * (VJP ? 4 : 2);
   const bool in_smem = fixed + state_bytes <= kMaxDynSmem;
   const size_t smem = fixed + (in_smem ? state_bytes : 0);
@@ -230,6 +251,9 @@ int run_sweep(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   if (rc != BCJR_OK) return rc;
 
   const size_t SV = (size_t)sh.S * sh.V;
+  cap_grid_by_memory(&grid, sizeof(float) * (size_t)sh.n * sh.J * (VJP ? 2 : 1) + sizeof(double) * sh.n +
+                                (in_smem ? 0 : sizeof(float) * 4 * (size_t)sh.J) +
+                                (VJP ? (sizeof(float) + sizeof(double)) * SV : 0));
   auto layout = [&](Arena& ar, SweepParams& P) {
     P.cs = ar.take<float>(SV);
     P.hist_l = ar.take<float>((size_t)grid * sh.n * sh.J);
@@ -326,6 +350,7 @@ int run_viterbi(const Shape& sh, const float* w, const float* c, int32_t* out_st
   int grid = 0;
   int rc = grid_for(kern, threads, smem, sh.n_seq, &grid);
   if (rc != BCJR_OK) return rc;
+  cap_grid_by_memory(&grid, (size_t)sh.n * sh.J + (in_smem ? 0 : sizeof(float) * 2 * (size_t)sh.J));
   ViterbiParams P{};
   auto layout = [&](Arena& ar) {
     P.bp = ar.take<uint8_t>((size_t)grid * sh.n * sh.J);

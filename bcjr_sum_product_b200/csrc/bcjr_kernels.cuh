@@ -114,6 +114,8 @@ __global__ void __launch_bounds__(kMaxThreads) bcjr_sweep_kernel(SweepParams P) 
   constexpr int B = 1 << D;
   constexpr bool VJP = (MODE == MODE_VJP);
   constexpr int NP = V + 1;
+  // VJP: three more per-warp partials per step, sum P(i) (A + Bc), sum P(i) Bc, sum P(i)
+  constexpr int NPT = NP + (VJP ? 3 : 0);
   const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5;
   const int nwarps = (nthr + 31) >> 5;
   const int J = P.J, n = P.n, HI = P.L - D;
@@ -123,8 +125,8 @@ __global__ void __launch_bounds__(kMaxThreads) bcjr_sweep_kernel(SweepParams P) 
   float* wsc = smem;                                   // n*V scaled weights
   float* gsc = wsc + n * V;                            // n*V scaled upstream gradient (VJP)
   float* wmax = gsc + (VJP ? n * V : 0);               // [2][32]
-  float* part = wmax + 64;                             // [2][32][NP]
-  float* apart = part + 2 * 32 * NP;                   // [2][32] argmax value
+  float* part = wmax + 64;                             // [2][32][NPT]
+  float* apart = part + 2 * 32 * NPT;                  // [2][32] argmax value
   int* aidx = reinterpret_cast<int*>(apart + 64);      // [2][32] argmax index
   float* sbase = reinterpret_cast<float*>(aidx + 64);  // state buffers (if in smem)
   float* lb[2];
@@ -165,6 +167,9 @@ __global__ void __launch_bounds__(kMaxThreads) bcjr_sweep_kernel(SweepParams P) 
 #pragma unroll
       for (int v = 0; v < V; ++v) { wt[v] = wsc[t * V + v]; gt[v] = VJP ? gsc[t * V + v] : 0.f; }
       C += (double)R;
+      // A_{t-1} enters relative to its value at group 0 (stored values stay at
+      // the size of their spread over groups); the backward subtracts the same
+      const float rA = (VJP && t > 0) ? aprev[0] : 0.f;
       float tmax = -INFINITY;
       for (int j = tid; j < J; j += nthr) {
         float x[B], z[B];
@@ -183,7 +188,7 @@ __global__ void __launch_bounds__(kMaxThreads) bcjr_sweep_kernel(SweepParams P) 
             float h = 0.f;
 #pragma unroll
             for (int v = 0; v < V; ++v) h = fmaf(gt[v], c[v], h);
-            z[b] = ((t == 0) ? 0.f : aprev[s >> D]) + h;
+            z[b] = ((t == 0) ? 0.f : aprev[s >> D] - rA) + h;
           }
         }
         float sum = 0.f, num = 0.f;
@@ -234,7 +239,12 @@ __global__ void __launch_bounds__(kMaxThreads) bcjr_sweep_kernel(SweepParams P) 
       __syncthreads();
     }
     const float gzq = (VJP && P.gZ) ? P.gZ[seq] : 0.f;
-    const float hb = Hbar - gzq;  // G = p (A + h + Bc - hb)
+    // G_t(q) = p_t(q) (A_{t-1}(q >> D) + h_t(q) + Bc_t(q mod J) - K_t + gZ) with
+    // K_t = sum_j P_t(j) (A_t(j) + Bc_t(j)), P_t(j) the posterior of group j,
+    // formed from the same stored values one step earlier (K_{n-1} = Hbar), so
+    // that rounding carried along the recursions cancels in G.  Stored Bc_t is
+    // relative to rB, the posterior mean of the previous step's stored values.
+    float Kt = Hbar, rB = 0.f;
 
     // ------------------------------------------------------------ backward
     float Rr = 0.f;    // max of previous stored backward values
@@ -254,9 +264,11 @@ __global__ void __launch_bounds__(kMaxThreads) bcjr_sweep_kernel(SweepParams P) 
       const double Csig = (t >= 1) ? hist_c[t - 1] : 0.0;
       const float K = (float)(Csig + Cr - l2Z);
       const bool last = (t == n - 1);
-      float np_[NP];
+      const float rA = (VJP && t >= 1) ? hist_a[(size_t)(t - 1) * J] : 0.f;   // the forward's reference
+      const float hb = Kt + rA - rB - gzq;   // G = p (A + h + (Bc - rB) - hb)
+      float np_[NPT];
 #pragma unroll
-      for (int k2 = 0; k2 < NP; ++k2) np_[k2] = 0.f;
+      for (int k2 = 0; k2 < NPT; ++k2) np_[k2] = 0.f;
       float bestp = -1.f;
       int bestq = 0x7fffffff;
       float tmax = -INFINITY;
@@ -264,23 +276,33 @@ __global__ void __launch_bounds__(kMaxThreads) bcjr_sweep_kernel(SweepParams P) 
         const float lsig = (t >= 1) ? hist_l[(size_t)(t - 1) * J + i] : 0.f;
         float asig = 0.f;
         if constexpr (VJP) asig = (t >= 1) ? hist_a[(size_t)(t - 1) * J + i] : 0.f;
-        float y[B], z[B], cc[B][V];
+        // With more than 32 codeword components per group only the exponents
+        // stay live between the two member loops (codewords and suffix values
+        // are read again); up to 32 everything stays in registers.
+        constexpr bool RELOAD = (B * V > 32);
+        constexpr int BL = RELOAD ? 1 : B;
+        float y[B], z[BL], cc[BL][V];
         float m = -INFINITY;
 #pragma unroll
         for (int b = 0; b < B; ++b) {
           const int q = (i << D) | b;
-          load_cw<V>(cs, q, cc[b]);
+          float c[V];
+          load_cw<V>(cs, q, c);
           const int r = q & jmask;
           float acc = last ? 0.f : rcur[r];
 #pragma unroll
-          for (int v = 0; v < V; ++v) { float d = wt[v] - cc[b][v]; acc = fmaf(-d, d, acc); }
+          for (int v = 0; v < V; ++v) { float d = wt[v] - c[v]; acc = fmaf(-d, d, acc); }
           y[b] = acc;
           m = fmaxf(m, acc);
-          if constexpr (VJP) {
-            float h = 0.f;
+          if constexpr (!RELOAD) {
 #pragma unroll
-            for (int v = 0; v < V; ++v) h = fmaf(gt[v], cc[b][v], h);
-            z[b] = (last ? 0.f : bcur[r]) + h;
+            for (int v = 0; v < V; ++v) cc[b][v] = c[v];
+            if constexpr (VJP) {
+              float h = 0.f;
+#pragma unroll
+              for (int v = 0; v < V; ++v) h = fmaf(gt[v], c[v], h);
+              z[b] = (last ? 0.f : bcur[r] - rB) + h;
+            }
           }
         }
         const float gf = ex2f(m + lsig + K);  // posterior factor of the group
@@ -291,20 +313,34 @@ __global__ void __launch_bounds__(kMaxThreads) bcjr_sweep_kernel(SweepParams P) 
           sum += u;
           const float p = u * gf;
           const int q = (i << D) | b;
+          float c[V], zb = 0.f;
+          if constexpr (RELOAD) {
+            load_cw<V>(cs, q, c);
+            if constexpr (VJP) {
+              float h = 0.f;
+#pragma unroll
+              for (int v = 0; v < V; ++v) h = fmaf(gt[v], c[v], h);
+              zb = (last ? 0.f : bcur[q & jmask] - rB) + h;
+            }
+          } else {
+#pragma unroll
+            for (int v = 0; v < V; ++v) c[v] = cc[b][v];
+            if constexpr (VJP) zb = z[b];
+          }
           if constexpr (MODE == MODE_SOFT) {
 #pragma unroll
-            for (int v = 0; v < V; ++v) np_[v] = fmaf(p, cc[b][v], np_[v]);
+            for (int v = 0; v < V; ++v) np_[v] = fmaf(p, c[v], np_[v]);
             np_[V] += p;
             arg_better(bestp, bestq, p, q);
           } else {
-            num = fmaf(u, z[b], num);
-            const float G = p * (asig + z[b] - hb);
+            num = fmaf(u, zb, num);
+            const float G = p * (asig + zb - hb);
             np_[V] += G;
             float* gq = gc_seq + (size_t)q * V;
 #pragma unroll
             for (int v = 0; v < V; ++v) {
-              np_[v] = fmaf(G, cc[b][v], np_[v]);
-              const float d = wt[v] - cc[b][v];
+              np_[v] = fmaf(G, c[v], np_[v]);
+              const float d = wt[v] - c[v];
               float acc = fmaf(graw[v], p, gq[v]);
               gq[v] = fmaf(P.two_over_T / P.sk, G * d, acc);
             }
@@ -314,18 +350,25 @@ __global__ void __launch_bounds__(kMaxThreads) bcjr_sweep_kernel(SweepParams P) 
           const float l = m + lg2f(sum) - Rr;
           rnext[i] = l;
           tmax = fmaxf(tmax, l);
-          if constexpr (VJP) bnext[i] = __fdividef(num, sum);
+          if constexpr (VJP) {
+            const float bn = __fdividef(num, sum);
+            bnext[i] = bn;
+            const float pg = gf * sum;   // posterior of group i at step t-1
+            np_[NP] = fmaf(pg, asig + bn, np_[NP]);
+            np_[NP + 1] = fmaf(pg, bn, np_[NP + 1]);
+            np_[NP + 2] += pg;
+          }
         }
       }
       // per-warp partials of this step
 #pragma unroll
-      for (int k2 = 0; k2 < NP; ++k2) np_[k2] = warp_sum(np_[k2]);
+      for (int k2 = 0; k2 < NPT; ++k2) np_[k2] = warp_sum(np_[k2]);
       tmax = warp_max(tmax);
       if (MODE == MODE_SOFT) warp_argmax(bestp, bestq);
       const int pb = t & 1;
       if (lane == 0) {
 #pragma unroll
-        for (int k2 = 0; k2 < NP; ++k2) part[(pb * 32 + warp) * NP + k2] = np_[k2];
+        for (int k2 = 0; k2 < NPT; ++k2) part[(pb * 32 + warp) * NPT + k2] = np_[k2];
         wmax[pb * 32 + warp] = tmax;
         apart[pb * 32 + warp] = bestp;
         aidx[pb * 32 + warp] = bestq;
@@ -336,7 +379,7 @@ __global__ void __launch_bounds__(kMaxThreads) bcjr_sweep_kernel(SweepParams P) 
 #pragma unroll
         for (int k2 = 0; k2 < NP; ++k2) {
           float a = 0.f;
-          for (int w2 = 0; w2 < nwarps; ++w2) a += part[(pb * 32 + w2) * NP + k2];
+          for (int w2 = 0; w2 < nwarps; ++w2) a += part[(pb * 32 + w2) * NPT + k2];
           tot[k2] = a;
         }
         if constexpr (MODE == MODE_SOFT) {
@@ -360,6 +403,20 @@ __global__ void __launch_bounds__(kMaxThreads) bcjr_sweep_kernel(SweepParams P) 
       Cr += (double)Rr;
       Rr = -INFINITY;
       for (int w2 = 0; w2 < nwarps; ++w2) Rr = fmaxf(Rr, wmax[pb * 32 + w2]);
+      if constexpr (VJP) {
+        float sk_ = 0.f, sb_ = 0.f, sp_ = 0.f;
+        for (int w2 = 0; w2 < nwarps; ++w2) {
+          const float* r = part + (pb * 32 + w2) * NPT + NP;
+          sk_ += r[0]; sb_ += r[1]; sp_ += r[2];
+        }
+        Kt = sk_ / sp_;
+        rB = sb_ / sp_;
+        // sp_ = sum_q p_t(q): forward and backward carry different rounding
+        // relative to the one log Z, so the posterior sum drifts from 1 along
+        // the sweep; folding its logarithm into the backward offset
+        // renormalises every next step.
+        Cr -= (double)lg2f(sp_);
+      }
       // the next step overwrites the other parity only; this step's slots are
       // read above before any thread can pass the next barrier
     }

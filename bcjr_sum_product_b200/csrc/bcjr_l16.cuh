@@ -36,6 +36,7 @@ namespace l16 {
 constexpr int L = 16, D = 2, HB = 12;  // HB: bits of mid
 constexpr int J = 1 << 14, NMID = 1 << 12, NT = 512, KB = NMID / NT;
 constexpr int S = 1 << 16;
+static_assert(NT / 32 == 16, "the per-step reductions combine 16 warps");
 
 struct Params {
   const float* w;        // [n_seq][len]
@@ -163,6 +164,21 @@ __global__ void reduce_block_gc(const double* __restrict__ part, int nparts, flo
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
 __device__ __forceinline__ float2 f2s(float a) { return make_float2(a, a); }
 
+// Block-wide combination of the 16 per-warp partials of a step: lane l holds
+// warp (l mod 16)'s value and an xor butterfly over 16 lanes combines them.
+// Every level pairs lane l with l ^ o and both form the same commutative
+// result, so every lane of every warp ends with the same bits.
+__device__ __forceinline__ float bfly16_min(float v) {
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float bfly16_sum(float v) {
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
 template <bool ARGMAX>
 __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
   constexpr int NP = 2;
@@ -245,9 +261,7 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
       if (lane == 0) wmin[(t & 1) * 32 + warp] = tmin;
       if (tid == 0) hist_c[t] = C;
       __syncthreads();
-      Rn = INFINITY;
-#pragma unroll
-      for (int w2 = 0; w2 < nwarps; ++w2) Rn = fminf(Rn, wmin[(t & 1) * 32 + w2]);
+      Rn = bfly16_min(wmin[(t & 1) * 32 + (lane & 15)]);
     }
     // log2 Z = -Rn + log2 sum_j 2^(Rn - stored_j) + C
     double l2Z;
@@ -367,9 +381,7 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
         }
       }
       Cr -= (double)Rrn;
-      Rrn = INFINITY;
-#pragma unroll
-      for (int w2 = 0; w2 < nwarps; ++w2) Rrn = fminf(Rrn, wmin[pb * 32 + w2]);
+      Rrn = bfly16_min(wmin[pb * 32 + (lane & 15)]);
     }
     __syncthreads();
   }
@@ -393,18 +405,17 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
 // the backward loads one 16-byte vector of each per block.  The backward's Bc
 // ping-pongs in the same global scratch.
 __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
-  constexpr int NP = 2;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int nwarps = NT / 32;
   const int n = P.n;
 
   extern __shared__ __align__(16) float smem[];
   float* sb = smem;                                    // [2][J] negated state ping-pong
   float* lb[2] = {sb, sb + J};
-  float* wmin = sb + 2 * J;                            // [2][32]
-  float* part = wmin + 64;                             // [2][32][NP]
-  float* spare = part + 2 * 32 * NP;                   // [2][32] + [2][32] (unused)
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(spare + 128);  // [4]
+  // per-warp partials of a step, [2 parities][32][8]:
+  //   0: sum P(i) (A + Bc)   1: sum P(i) Bc   2: sum P(i)   3: min stored value
+  //   4: sum G c             5: sum G
+  float* rec = sb + 2 * J;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(rec + 2 * 32 * 8);  // [4]
   float* wsc = reinterpret_cast<float*>(tslot + 4);    // n: -w'
   float* gsc = wsc + n;                                // n: g / sk
 
@@ -448,6 +459,11 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
       float* acur = bcg[t & 1];
       const float2 nw2 = f2s(wsc[t]);
       const float2 g2 = f2s(gsc[t]);
+      // A_{t-1} enters relative to its value at group 0, so that the stored
+      // prefix expectations stay at the size of their spread over groups
+      // instead of growing with t; the histories keep the stored values and
+      // the backward subtracts the same reference.
+      const float2 nrA = f2s((t > 0) ? -aprev[0] : 0.f);
       C -= (double)Rn;
       float tmin = INFINITY;
       float apn[4] = {0.f, 0.f, 0.f, 0.f};
@@ -461,6 +477,7 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
         float cb[16];
         tmem_ld16(tbase + 16 * k, cb);
         const float2 ap01 = f2(apn[0], apn[1]), ap23 = f2(apn[2], apn[3]);
+        const float2 as01 = __fadd2_rn(ap01, nrA), as23 = __fadd2_rn(ap23, nrA);
         if (t > 0 && k + 1 < KB) {
 #pragma unroll
           for (int h = 0; h < 4; ++h) apn[h] = aprev[(h << HB) | (mid + NT)];
@@ -484,7 +501,7 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
           const float m = fminf(fminf(x01.x, x01.y), fminf(x23.x, x23.y));
           const float2 a01 = __ffma2_rn(x01, neg1, f2s(m)), a23 = __ffma2_rn(x23, neg1, f2s(m));
           const float2 u01 = f2(ex2f(a01.x), ex2f(a01.y)), u23 = f2(ex2f(a23.x), ex2f(a23.y));
-          const float2 z01 = __ffma2_rn(g2, c01, ap01), z23 = __ffma2_rn(g2, c23, ap23);
+          const float2 z01 = __ffma2_rn(g2, c01, as01), z23 = __ffma2_rn(g2, c23, as23);
           const float2 s2 = __fadd2_rn(u01, u23);
           const float2 q2 = __ffma2_rn(u23, z23, __fmul2_rn(u01, z01));
           const float ssum = s2.x + s2.y;
@@ -496,12 +513,10 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
         reinterpret_cast<float4*>(acur)[mid] = make_float4(aout[0], aout[1], aout[2], aout[3]);
       }
       tmin = -warp_max(-tmin);
-      if (lane == 0) wmin[(t & 1) * 32 + warp] = tmin;
+      if (lane == 0) rec[((t & 1) * 32 + warp) * 8 + 3] = tmin;
       if (tid == 0) hist_c[t] = C;
       __syncthreads();
-      Rn = INFINITY;
-#pragma unroll
-      for (int w2 = 0; w2 < nwarps; ++w2) Rn = fminf(Rn, wmin[(t & 1) * 32 + w2]);
+      Rn = bfly16_min(rec[((t & 1) * 32 + (lane & 15)) * 8 + 3]);
     }
     // log2 Z and Hbar = E[A_{n-1}]
     double l2Z;
@@ -517,16 +532,15 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
       }
       s0 = warp_sum(s0);
       s1 = warp_sum(s1);
-      if (lane == 0) { part[warp * NP] = s0; part[warp * NP + 1] = s1; }
+      if (lane == 0) { rec[warp * 8 + 4] = s0; rec[warp * 8 + 5] = s1; }
       __syncthreads();
-      float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-      for (int w2 = 0; w2 < nwarps; ++w2) { a0 += part[w2 * NP]; a1 += part[w2 * NP + 1]; }
+      const float a0 = bfly16_sum(rec[(lane & 15) * 8 + 4]);
+      const float a1 = bfly16_sum(rec[(lane & 15) * 8 + 5]);
       l2Z = -(double)Rn + log2((double)a0) + C;
       Hbar = a1 / a0;
       __syncthreads();
     }
-    const float hb = Hbar - (P.gZ ? P.gZ[seq] : 0.f);
+    const float gzq = P.gZ ? P.gZ[seq] : 0.f;
     const float2 nc2T = f2s(-P.two_over_T / P.sk);
 
     // tensor memory now accumulates this sequence's codebook gradient
@@ -544,6 +558,12 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
     // columns; codewords and history values are prefetched one unit ahead.
     float Rrn = 0.f;
     double Cr = 0.0;
+    // G_t(q) = p_t(q) (A_{t-1}(q >> 2) + h_t(q) + Bc_t(q mod J) - K_t + gZ) with
+    // K_t = sum_j P_t(j) (A_t(j) + Bc_t(j)), P_t(j) the posterior of group j,
+    // formed from the same stored values one step earlier (K_{n-1} = Hbar), so
+    // that rounding carried along the recursions cancels in G.  Stored Bc_t is
+    // relative to rB, the posterior mean of the previous step's stored values.
+    float Kt = Hbar, rB = 0.f;
     float cbn[8], cbm[8];
     ld_cb8(cs_tm, tid, 0, cbn);
     ld_cb8(cs_tm, tid, 1, cbm);
@@ -565,7 +585,10 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
       const double Csig = (t >= 1) ? hist_c[t - 1] : 0.0;
       const float K = (float)(Csig + Cr - l2Z);
       const bool last = (t == n - 1);
+      const float rA = (t >= 1) ? hist_a[(size_t)(t - 1) * J] : 0.f;   // the forward's reference
+      const float hbt = Kt + rA - rB - gzq;
       float2 accG = f2s(0.f), accGc = f2s(0.f);
+      float2 accK = f2s(0.f), accB = f2s(0.f), accP = f2s(0.f);
       float tmin = INFINITY;
       float4 bvn = make_float4(0.f, 0.f, 0.f, 0.f);
       if (!last) bvn = reinterpret_cast<const float4*>(bcur)[tid];
@@ -579,7 +602,7 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
         } else {
           const float4 rv = reinterpret_cast<const float4*>(ncur)[mid];
           nr[0] = rv.x; nr[1] = rv.y; nr[2] = rv.z; nr[3] = rv.w;
-          bc[0] = bvn.x; bc[1] = bvn.y; bc[2] = bvn.z; bc[3] = bvn.w;
+          bc[0] = bvn.x - rB; bc[1] = bvn.y - rB; bc[2] = bvn.z - rB; bc[3] = bvn.w - rB;
         }
         if (!last && k + 1 < KB) bvn = reinterpret_cast<const float4*>(bcur)[mid + NT];
         const float4 hs4 = hsn, ha4 = han;
@@ -614,7 +637,7 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
                               fminf(fminf(y[0].y, y[1].y), fminf(y[2].y, y[3].y)));
           const float2 ge = __fadd2_rn(__fadd2_rn(f2s(K), f2(-hs0, -hs1)), __fmul2_rn(m, neg1));
           const float2 gf = f2(ex2f(ge.x), ex2f(ge.y));
-          const float2 ah = f2(ha0 - hb, ha1 - hb);   // A - Hbar + gZ
+          const float2 ah = f2(ha0 - hbt, ha1 - hbt);   // A - K + gZ
           float2 ssum = f2s(0.f), num = f2s(0.f);
 #pragma unroll
           for (int lo = 0; lo < 4; ++lo) {
@@ -638,6 +661,11 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
           nout[2 * g + 1] = (m.y - Rrn) - lg2f(ssum.y);
           bout[2 * g] = __fdividef(num.x, ssum.x);
           bout[2 * g + 1] = __fdividef(num.y, ssum.y);
+          // posterior of the two step t-1 groups, P(i) = sum_lo p
+          const float2 pg = __fmul2_rn(gf, ssum), bo = f2(bout[2 * g], bout[2 * g + 1]);
+          accK = __ffma2_rn(pg, __fadd2_rn(f2(ha0, ha1), bo), accK);
+          accB = __ffma2_rn(pg, bo, accB);
+          accP = __fadd2_rn(accP, pg);
         }
         if (t >= 1) {
 #pragma unroll
@@ -651,25 +679,37 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
       tmem_wait_st();
       const float a0 = warp_sum(accGc.x + accGc.y);
       const float a1 = warp_sum(accG.x + accG.y);
+      const float kk = warp_sum(accK.x + accK.y);
+      const float kb = warp_sum(accB.x + accB.y);
+      const float kp = warp_sum(accP.x + accP.y);
       tmin = -warp_max(-tmin);
       const int pb = t & 1;
       if (lane == 0) {
-        part[(pb * 32 + warp) * NP] = a0;
-        part[(pb * 32 + warp) * NP + 1] = a1;
-        wmin[pb * 32 + warp] = tmin;
+        float* r = rec + (pb * 32 + warp) * 8;
+        *reinterpret_cast<float4*>(r) = make_float4(kk, kb, kp, tmin);
+        r[4] = a0;
+        r[5] = a1;
       }
       __syncthreads();
       if (tid == 0) {
         float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-        for (int w2 = 0; w2 < nwarps; ++w2) { s0 += part[(pb * 32 + w2) * NP]; s1 += part[(pb * 32 + w2) * NP + 1]; }
+        for (int w2 = 0; w2 < NT / 32; ++w2) { s0 += rec[(pb * 32 + w2) * 8 + 4]; s1 += rec[(pb * 32 + w2) * 8 + 5]; }
         // dl/dw_t = (2/T) (sum G c - w_t sum G), c = c'/sk, w_t = -nwt/sk
         P.grad_w[seq * P.len + t] = P.two_over_T * (s0 + nwt * s1) / P.sk;
       }
       Cr -= (double)Rrn;
-      Rrn = INFINITY;
-#pragma unroll
-      for (int w2 = 0; w2 < nwarps; ++w2) Rrn = fminf(Rrn, wmin[pb * 32 + w2]);
+      {
+        const float4 r = *reinterpret_cast<const float4*>(rec + (pb * 32 + (lane & 15)) * 8);
+        const float sp = bfly16_sum(r.z);   // sum_q p_t(q), 1 up to rounding
+        Kt = bfly16_sum(r.x) / sp;
+        rB = bfly16_sum(r.y) / sp;
+        Rrn = bfly16_min(r.w);
+        // Forward and backward carry different rounding relative to the one
+        // log Z, so the posterior sum drifts from 1 along the sweep; folding
+        // its logarithm into the backward offset renormalises every next step.
+        Cr -= (double)lg2f(sp);
+      }
     }
 
     // fold this sequence's codebook gradient into the CTA partial

@@ -190,3 +190,36 @@ def test_l16_viterbi_matches_generic_and_oracle(monkeypatch):
     ref = oracle.viterbi(w[:6], c, 16, 2, 1)
     np.testing.assert_array_equal(s_fast[:6].cpu().numpy(), ref["states"])
     np.testing.assert_array_equal(c_fast[:6].cpu().numpy(), ref["cost"])
+
+
+def test_longest_sequences(monkeypatch):
+    """len = 8192 (the largest supported): L=12 against the oracle, and L=16
+    (whose per-CTA histories are 0.5-1 GB, so fewer CTAs are resident) against
+    the generic kernels."""
+    w, c, g = I.random_case(12, 2, 1, 3, 8192, seed=777)
+    gpu = _run_all(w, c, 12, 2, 1, 0.2, g, torch.zeros(3))
+    _compare(w, c, 12, 2, 1, 0.2, g, torch.zeros(3), gpu)
+    # an upstream gradient with a non-zero mean makes the prefix and suffix
+    # expectations grow linearly along the sequence
+    gb = g[:1] + 1.0
+    gpu = _run_all(w[:1], c, 12, 2, 1, 0.05, gb, torch.ones(1))
+    _compare(w[:1], c, 12, 2, 1, 0.05, gb, torch.ones(1), gpu)
+    # at T = 0.01 the posterior of a near tie depends on log values of a few
+    # hundred, whose fp32 rounding differs between the two sweeps
+    w, c, g = I.random_case(10, 2, 1, 1, 8192, seed=9)
+    gb = g + 1.0
+    gpu = _run_all(w, c, 10, 2, 1, 0.01, gb, torch.ones(1))
+    _compare(w, c, 10, 2, 1, 0.01, gb, torch.ones(1), gpu)
+    w, c, g = I.random_case(16, 2, 1, 2, 8192, seed=778)
+    g[1] += 1.0
+    wd, cd, gd = w.to(DEV), c.to(DEV), g.to(DEV)
+    fast = [x.cpu().numpy() for x in lib.soft_codeword(wd, cd, 16, 2, 1, 0.1) + lib.vjp(wd, cd, 16, 2, 1, 0.1, gd)]
+    vs_fast = lib.viterbi_decode(wd, cd, 16, 2, 1)[0].cpu()
+    monkeypatch.setenv("BCJR_GENERIC_ONLY", "1")
+    gen = [x.cpu().numpy() for x in lib.soft_codeword(wd, cd, 16, 2, 1, 0.1) + lib.vjp(wd, cd, 16, 2, 1, 0.1, gd)]
+    vs_gen = lib.viterbi_decode(wd, cd, 16, 2, 1)[0].cpu()
+    assert_soft(fast[0], gen[0], c)
+    assert_logZ(fast[1], gen[1], 16, 2, 8192)
+    assert_grad(fast[2], gen[2], "grad_w")
+    assert_grad(fast[3], gen[3], "grad_c")
+    assert torch.equal(vs_fast, vs_gen)
