@@ -373,7 +373,7 @@ int run_viterbi(const Shape& sh, const float* w, const float* c, int32_t* out_st
   return BCJR_OK;
 }
 
-__device__ int g_device_error = 0;
+static_assert(bcjr::kErrTimeout == BCJR_ERR_TIMEOUT, "device and host status codes agree");
 
 }  // namespace
 
@@ -447,8 +447,8 @@ int bcjr_get_device_error(void* stream) {
     return BCJR_ERR_CUDA;
   }
   int flag = 0, zero = 0;
-  if (cudaMemcpyFromSymbol(&flag, g_device_error, sizeof(int)) != cudaSuccess) return BCJR_ERR_CUDA;
-  if (flag != 0 && cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return BCJR_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&flag, bcjr::g_device_error, sizeof(int)) != cudaSuccess) return BCJR_ERR_CUDA;
+  if (flag != 0 && cudaMemcpyToSymbol(bcjr::g_device_error, &zero, sizeof(int)) != cudaSuccess) return BCJR_ERR_CUDA;
   return flag;
 }
 

@@ -38,6 +38,12 @@ namespace bcjr {
 constexpr int kMaxThreads = 512;
 constexpr int kMaxWarps = kMaxThreads / 32;
 
+// First device-side error recorded by a kernel of this library (a status code
+// of the C interface, 0 = none); read and cleared by bcjr_get_device_error.
+__device__ int g_device_error = 0;
+constexpr int kErrTimeout = 4;   // a bounded wait ran out
+__device__ __forceinline__ void record_device_error(int code) { atomicCAS(&g_device_error, 0, code); }
+
 struct SweepParams {
   const float* w;        // [n_seq][len]
   const float* cs;       // scaled codebook c' [S][V]

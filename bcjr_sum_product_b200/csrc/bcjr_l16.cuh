@@ -118,6 +118,21 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&r)[8]) {
 
 __host__ __device__ constexpr int bidx(int h, int lo) { return 8 * (h >> 1) + 2 * lo + (h & 1); }
 
+// Bulk prefetch of `bytes` (a multiple of 16, 16-byte aligned) from global
+// memory into L2 by the tensor-memory-access unit: no registers, no shared
+// memory, nothing to wait for.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+// The backward of step t reads the history of step t - 1; at its start lanes
+// 0..7 of one warp ask for step t - 2's (64 KB, eight 8 KB blocks) so that it is
+// in L2, not HBM, when the per-thread loads of the next step are issued.
+__device__ __forceinline__ void prefetch_history(const float* hist, int t, int lane) {
+  constexpr uint32_t kChunk = J * sizeof(float) / 8;
+  if (t >= 2 && lane < 8)
+    prefetch_l2_bulk(reinterpret_cast<const char*>(hist + (size_t)(t - 2) * J) + lane * kChunk, kChunk);
+}
+
 __device__ __forceinline__ void ld_cb(const float* __restrict__ cs_tm, int mid, float (&c)[16]) {
   const float4* p = reinterpret_cast<const float4*>(cs_tm + (size_t)mid * 16);
 #pragma unroll
@@ -290,6 +305,7 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
     };
     float4 hsn = hist_at(n - 1, 0), hsm = hist_at(n - 1, 1);
     for (int t = n - 1; t >= 0; --t) {
+      if (warp == 0) prefetch_history(hist, t, lane);
       const float* ncur = lb[t & 1];
       float* nnext = lb[(t + 1) & 1];
       const float2 nw2 = f2s(wsc[t]);
