@@ -11,6 +11,12 @@ seed 2).  Metric: state-updates/s = n_seq * n_steps * 2^L per step / time
 (weights/s reported alongside).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload qtip|mid|mlp|layer|tiny] [--temp T]
+
+The default workload is the QTIP-scale one above.  ``--workload`` measures the
+other seeded workloads of the inputs module with the same timing rules (``mid``
+is forward only: soft codeword and logZ; ``mlp`` takes ``--temp`` from
+{1, 0.1, 0.01}).
 
 N > 1 runs under torch.distributed.run, one rank per GPU, each rank on its own
 copy of the workload (weak scaling); the codebook gradient is summed across
@@ -35,13 +41,19 @@ METRIC = "BCJR state-updates/s and weights/s (fwd+bwd+VJP) at L=16 k=2, 1 B200"
 UNIT = "state-updates/s"
 WORKLOAD = "qtip"
 
-# Algorithmic work per (sequence, step, state) unit for k=2, V=1 (B = 4),
-# fixed before optimisation (FP32-pipe ops, MUFU ex2 ops); recomputation and
-# ALU-pipe work (max, compares, address arithmetic) are not counted.
-LEDGER = {
-    "soft": {"fp32": 3.75 + 6.75, "mufu": 2.0},
-    "vjp": {"fp32": 7.5 + 16.5, "mufu": 2.0},
+# Algorithmic work per (sequence, step, state) unit, fixed before optimisation
+# (FP32-pipe ops, MUFU ex2 ops of a linear-domain sweep with one ex2 per state
+# per sweep); recomputation and ALU-pipe work (max, compares, address
+# arithmetic) are not counted.  k=2, V=1 (B = 4): forward 3.75 (energy FFMA,
+# 0.75 gather FADD, rescale, psi*u), backward + posterior + soft codeword 6.75,
+# VJP forward 7.5, VJP backward + G + gradients 16.5.  k=2, V=2 (B = 16): the
+# energy, h = g.c and each gradient term take one op per component and the
+# gather 15/16 per state: 4.94, 8.94, 10.88, 22.69.
+LEDGERS = {
+    (2, 1): {"soft": {"fp32": 3.75 + 6.75, "mufu": 2.0}, "vjp": {"fp32": 7.5 + 16.5, "mufu": 2.0}},
+    (2, 2): {"soft": {"fp32": 4.94 + 8.94, "mufu": 2.0}, "vjp": {"fp32": 10.88 + 22.69, "mufu": 2.0}},
 }
+LEDGER = LEDGERS[(2, 1)]
 # DRAM bytes per sequence (read + write) of each L=16 sweep kernel, from one
 # ncu capture of 16 qtip sequences (profiles/vjp_kernel_qtip16.md,
 # profiles/soft_kernel_qtip16.md); set to None whenever the kernel changes.
@@ -51,9 +63,10 @@ MUFU_PER_CLK_SM = 16.0    # ex2 per SM per clock (measured 15.99 on this machine)
 N_SM = 148
 
 
-def peak_units_per_s(kind: str, mhz: float) -> float:
-    led = LEDGER[kind] if kind != "step" else {
-        "fp32": LEDGER["soft"]["fp32"] + LEDGER["vjp"]["fp32"], "mufu": LEDGER["soft"]["mufu"] + LEDGER["vjp"]["mufu"]}
+def peak_units_per_s(kind: str, mhz: float, ledger=None) -> float:
+    ledger = ledger or LEDGER
+    led = ledger[kind] if kind != "step" else {
+        "fp32": ledger["soft"]["fp32"] + ledger["vjp"]["fp32"], "mufu": ledger["soft"]["mufu"] + ledger["vjp"]["mufu"]}
     clk_per_unit = max(led["fp32"] / FP32_PER_CLK_SM, led["mufu"] / MUFU_PER_CLK_SM)
     return N_SM * mhz * 1e6 / clk_per_unit
 
@@ -112,21 +125,36 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def cpu_baseline(wl, inp, n_rows: int):
+def cpu_baseline(wl, inp, n_rows: int, T: float, do_vjp: bool):
     """The oracle as it stands, on n_rows sequences of the workload, all host cores."""
     import oracle
     cores = os.cpu_count() or 1
     rows = list(range(n_rows))
-    w, g = inp.w[rows].contiguous(), inp.g[rows].contiguous()
-    T = wl.temps[0]
+    w = inp.w[rows].contiguous()
     t0 = time.perf_counter()
     oracle.soft(w, inp.c, wl.L, wl.k, wl.V, T, nthreads=cores)
-    oracle.vjp(w, inp.c, wl.L, wl.k, wl.V, T, g, nthreads=cores)
+    if do_vjp:
+        oracle.vjp(w, inp.c, wl.L, wl.k, wl.V, T, inp.g[rows].contiguous(), nthreads=cores)
     dt = time.perf_counter() - t0
     units = n_rows * wl.n_steps * wl.S
+    what = "soft codeword + VJP" if do_vjp else "soft codeword"
     return {"value": units / dt, "unit": UNIT, "cores": min(cores, n_rows), "kind": "oracle",
-            "sample": f"{n_rows} of {wl.n_seq} sequences of the {wl.name} workload, soft codeword + VJP, "
+            "sample": f"{n_rows} of {wl.n_seq} sequences of the {wl.name} workload, {what}, "
                       f"fp64 C oracle with OpenMP over sequences; {dt:.1f} s"}
+
+
+def describe(wl, T: float, do_vjp: bool) -> str:
+    mats = ", ".join(f"{r}x{c}" for r, c in wl.matrices)
+    what = "soft codeword + logZ + VJP" if do_vjp else "soft codeword + logZ"
+    return (f"{wl.name}: L={wl.L} k={wl.k} V={wl.V}, fp32 matrices {mats} as {wl.n_seq} x {wl.seq_len}-weight "
+            f"sequences ({wl.n_steps} steps), T={T:g}, {what} per step")
+
+
+def metric_for(wl, do_vjp: bool) -> str:
+    if wl.name == WORKLOAD:
+        return METRIC
+    return (f"BCJR state-updates/s and weights/s ({'fwd+bwd+VJP' if do_vjp else 'fwd+bwd'}) on the {wl.name} "
+            f"workload (L={wl.L} k={wl.k} V={wl.V}), 1 B200")
 
 
 def run_reference(args):
@@ -135,16 +163,18 @@ def run_reference(args):
     if rank != 0:
         return 0
     from bcjr_sum_product_b200 import inputs as I
-    wl = I.WORKLOADS[WORKLOAD]
+    wl = I.WORKLOADS[args.workload]
+    T = args.temp if args.temp is not None else wl.temps[0]
+    do_vjp = "vjp" in wl.calls
     cores = os.cpu_count() or 1
-    n_rows = max(1, min(cores, 16))
-    inp = I.make(WORKLOAD, rows=list(range(n_rows)))
+    n_rows = max(1, min(cores, 16, wl.n_seq))
+    inp = I.make(args.workload, rows=list(range(n_rows)))
     import oracle
-    T = wl.temps[0]
 
     def step():
         oracle.soft(inp.w, inp.c, wl.L, wl.k, wl.V, T, nthreads=cores)
-        oracle.vjp(inp.w, inp.c, wl.L, wl.k, wl.V, T, inp.g, nthreads=cores)
+        if do_vjp:
+            oracle.vjp(inp.w, inp.c, wl.L, wl.k, wl.V, T, inp.g, nthreads=cores)
 
     for _ in range(args.warmup):
         step()
@@ -154,12 +184,12 @@ def run_reference(args):
     dt = (time.perf_counter() - t0) / max(1, args.steps)
     units = n_rows * wl.n_steps * wl.S
     value = units / dt
-    sample = f"{n_rows} of {wl.n_seq} sequences of the {wl.name} workload per step (soft codeword + VJP)"
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"{wl.name}: L=16 k=2 V=1, 2048x2048 fp32 matrix as {wl.n_seq} x 256-weight "
-                                   f"sequences, T=0.05, soft codeword + logZ + VJP", "sample_sequences": n_rows},
+    sample = (f"{n_rows} of {wl.n_seq} sequences of the {wl.name} workload per step "
+              f"({'soft codeword + VJP' if do_vjp else 'soft codeword'})")
+    line = {"impl": "reference", "metric": metric_for(wl, do_vjp), "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": describe(wl, T, do_vjp), "sample_sequences": n_rows},
             "weights_per_s": n_rows * wl.seq_len / dt,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(cores, n_rows), "kind": "oracle",
                              "sample": sample},
@@ -178,7 +208,12 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seqs", type=int, default=0,
                     help="profiling only: run on the first N sequences of the workload (not a bench number)")
+    ap.add_argument("--workload", default=WORKLOAD, choices=["qtip", "mid", "mlp", "layer", "tiny"])
+    ap.add_argument("--temp", type=float, default=None, help="temperature (one of the workload's)")
     args = ap.parse_args()
+    from bcjr_sum_product_b200 import inputs as I
+    if args.temp is not None and args.temp not in I.WORKLOADS[args.workload].temps:
+        ap.error(f"--temp must be one of {I.WORKLOADS[args.workload].temps}")
     if args.impl == "reference":
         return run_reference(args)
 
@@ -199,13 +234,15 @@ def main():
     torch.cuda.set_device(dev)
     lib.load()
 
-    wl = I.WORKLOADS[WORKLOAD]
-    inp = I.make(WORKLOAD, rows=list(range(args.seqs)) if args.seqs > 0 else None)
-    T = wl.temps[0]
+    wl = I.WORKLOADS[args.workload]
+    do_vjp = "vjp" in wl.calls
+    inp = I.make(args.workload, rows=list(range(args.seqs)) if args.seqs > 0 else None, with_grad=do_vjp)
+    T = args.temp if args.temp is not None else wl.temps[0]
     L, k, V = wl.L, wl.k, wl.V
+    ledger = LEDGERS.get((k, V))
     n_seq = inp.w.shape[0]
     stream = torch.cuda.current_stream(dev)
-    w = inp.w.to(dev); c = inp.c.to(dev); g = inp.g.to(dev)
+    w = inp.w.to(dev); c = inp.c.to(dev); g = inp.g.to(dev) if do_vjp else None
     soft = torch.empty_like(w); logZ = torch.empty(n_seq, device=dev)
     gw = torch.empty_like(w); gc = torch.empty_like(c)
     flush = torch.empty(256 * 1024 * 1024 // 4, device=dev)  # 256 MB > 126 MB L2
@@ -216,7 +253,8 @@ def main():
     def step():
         lib.soft_codeword(w, c, L, k, V, T, out_soft=soft, out_logZ=logZ, stream=stream)
         # each rank: VJP of its own sequences, then the codebook gradient summed over ranks
-        bdist.vjp_data_parallel(local_vjp, w, c, g)
+        if do_vjp:
+            bdist.vjp_data_parallel(local_vjp, w, c, g)
 
     for _ in range(args.warmup):
         step()
@@ -237,7 +275,8 @@ def main():
         e0.record(stream)
         lib.soft_codeword(w, c, L, k, V, T, out_soft=soft, out_logZ=logZ, stream=stream)
         e1.record(stream)
-        bdist.vjp_data_parallel(local_vjp, w, c, g)
+        if do_vjp:
+            bdist.vjp_data_parallel(local_vjp, w, c, g)
         e2.record(stream)
         e2.synchronize()
         soft_ms.append(e0.elapsed_time(e1)); vjp_ms.append(e1.elapsed_time(e2)); step_ms.append(e0.elapsed_time(e2))
@@ -260,22 +299,29 @@ def main():
     # e2e: through the public API with host buffers, copies inside the timed region
     e2e = None
     if not args.no_e2e:
-        hw = inp.w.pin_memory(); hc = inp.c.pin_memory(); hg = inp.g.pin_memory()
+        hw = inp.w.pin_memory(); hc = inp.c.pin_memory(); hg = inp.g.pin_memory() if do_vjp else None
         out_soft_h = torch.empty_like(hw).pin_memory(); out_logZ_h = torch.empty(n_seq).pin_memory()
-        out_gw_h = torch.empty_like(hw).pin_memory(); out_gc_h = torch.empty_like(hc).pin_memory()
-        h2d = hw.numel() * 4 + hc.numel() * 4 + hg.numel() * 4
-        d2h = out_soft_h.numel() * 4 + out_logZ_h.numel() * 4 + out_gw_h.numel() * 4 + out_gc_h.numel() * 4
+        out_gw_h = torch.empty_like(hw).pin_memory() if do_vjp else None
+        out_gc_h = torch.empty_like(hc).pin_memory() if do_vjp else None
+        h2d = hw.numel() * 4 + hc.numel() * 4 + (hg.numel() * 4 if do_vjp else 0)
+        d2h = out_soft_h.numel() * 4 + out_logZ_h.numel() * 4
+        if do_vjp:
+            d2h += out_gw_h.numel() * 4 + out_gc_h.numel() * 4
         k_e2e = max(1, min(args.steps, 3))
         times = []
         for _ in range(k_e2e):
             flush.fill_(1.0)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            w.copy_(hw, non_blocking=True); c.copy_(hc, non_blocking=True); g.copy_(hg, non_blocking=True)
+            w.copy_(hw, non_blocking=True); c.copy_(hc, non_blocking=True)
+            if do_vjp:
+                g.copy_(hg, non_blocking=True)
             lib.soft_codeword(w, c, L, k, V, T, out_soft=soft, out_logZ=logZ, stream=stream)
-            bdist.vjp_data_parallel(local_vjp, w, c, g)
+            if do_vjp:
+                bdist.vjp_data_parallel(local_vjp, w, c, g)
             out_soft_h.copy_(soft, non_blocking=True); out_logZ_h.copy_(logZ, non_blocking=True)
-            out_gw_h.copy_(gw, non_blocking=True); out_gc_h.copy_(gc, non_blocking=True)
+            if do_vjp:
+                out_gw_h.copy_(gw, non_blocking=True); out_gc_h.copy_(gc, non_blocking=True)
             b.record(stream)
             b.synchronize()
             times.append(a.elapsed_time(b))
@@ -293,19 +339,25 @@ def main():
 
     peaks, basis = measured_peaks()
     fmax = float(peaks.get("sm_max_mhz", 1965.0))
-    dominant = "vjp" if ms_vjp >= ms_soft else "soft"
+    dominant = "vjp" if do_vjp and ms_vjp >= ms_soft else "soft"
     ms_dom = ms_vjp if dominant == "vjp" else ms_soft
     achieved = units / (ms_dom / 1e3)
-    peak = peak_units_per_s(dominant, fmax)
-    tps = TRAFFIC_PER_SEQ.get(dominant)
-    roofline = {"bound": "alu", "kernel": f"bcjr::l16::{dominant}_kernel", "achieved": achieved, "peak": peak,
-                "unit": UNIT, "frac": achieved / peak, "traffic": (tps * n_seq) if tps else None,
-                "traffic_note": "DRAM bytes per launch, scaled from an ncu capture of 16 sequences",
-                "peak_basis": f"{N_SM} SMs x min(128 FP32 / {LEDGER[dominant]['fp32']}, 16 MUFU / "
-                              f"{LEDGER[dominant]['mufu']}) units/clk at sm_max {fmax:.0f} MHz ({basis})",
-                "step_frac": value / world / peak_units_per_s("step", fmax)}
-    if clocks.get("sm_mhz"):
-        roofline["frac_at_sampled_clock"] = achieved / peak_units_per_s(dominant, clocks["sm_mhz"])
+    block_layout = (L, k, V) == (16, 2, 1)
+    kernel = (f"bcjr::l16::{dominant}_kernel" if block_layout else
+              f"bcjr::bcjr_sweep_kernel<{V},{k * V},{1 if dominant == 'vjp' else 0}>")
+    roofline = None
+    if ledger is not None:
+        peak = peak_units_per_s(dominant, fmax, ledger)
+        tps = TRAFFIC_PER_SEQ.get(dominant) if block_layout else None
+        roofline = {"bound": "alu", "kernel": kernel, "achieved": achieved, "peak": peak,
+                    "unit": UNIT, "frac": achieved / peak, "traffic": (tps * n_seq) if tps else None,
+                    "traffic_note": "DRAM bytes per launch, scaled from an ncu capture of 16 sequences",
+                    "peak_basis": f"{N_SM} SMs x min(128 FP32 / {ledger[dominant]['fp32']}, 16 MUFU / "
+                                  f"{ledger[dominant]['mufu']}) units/clk at sm_max {fmax:.0f} MHz ({basis})"}
+        if do_vjp:
+            roofline["step_frac"] = value / world / peak_units_per_s("step", fmax, ledger)
+        if clocks.get("sm_mhz"):
+            roofline["frac_at_sampled_clock"] = achieved / peak_units_per_s(dominant, clocks["sm_mhz"], ledger)
 
     cpu = None
     if args.seqs > 0:
@@ -314,20 +366,19 @@ def main():
         line_note = None
     if world == 1 and not args.no_cpu_baseline:
         cores = os.cpu_count() or 1
-        cpu = cpu_baseline(wl, inp, max(1, min(cores, 16, n_seq)))
+        cpu = cpu_baseline(wl, inp, max(1, min(cores, 16, n_seq)), T, do_vjp)
 
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+    line = {"metric": metric_for(wl, do_vjp), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": f"{wl.name}: L=16 k=2 V=1, 2048x2048 fp32 matrix as {wl.n_seq} x 256-weight "
-                                   f"sequences, T=0.05, soft codeword + logZ + VJP per step",
+            "config": {"workload": describe(wl, T, do_vjp),
                        "n_seq_per_gpu": n_seq, "steps_per_seq": wl.n_steps, "states": wl.S,
                        "l2": "flushed between timed iterations (256 MB write outside the events)",
                        "parallelism": f"dp{world}" if world > 1 else "single"},
             "weights_per_s": world * n_seq * wl.seq_len / (ms_step / 1e3),
             "ms_soft": ms_soft, "ms_vjp": ms_vjp, "wall_s": wall,
             "ms_step_min_max": [min(step_ms), max(step_ms)],
-            "gpu_launches": 5 * args.steps,
+            "gpu_launches": (5 if do_vjp else 2) * args.steps,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks}
     if line_note:
         line["note"] = line_note
