@@ -11,6 +11,7 @@
 #include "bcjr.h"
 #include "bcjr_kernels.cuh"
 #include "bcjr_l16.cuh"
+#include "bcjr_l16v2.cuh"
 
 namespace {
 
@@ -232,11 +233,61 @@ int run_l16(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
 }
 
 bool use_l16(const Shape& sh) { return !generic_only() && sh.L == 16 && sh.D == 2 && sh.V == 1; }
+bool use_l16v2(const Shape& sh) { return !generic_only() && sh.L == 16 && sh.D == 4 && sh.V == 2; }
+
+// L = 16, k = 2, V = 2: the kernels of bcjr_l16v2.cuh.
+template <int MODE>
+int run_l16v2(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
+  namespace K = bcjr::l16v2;
+  constexpr bool VJP = MODE == bcjr::MODE_VJP;
+  void (*kern)(K::Params) = K::vjp_kernel;
+  if (!VJP) kern = a.out_argmax ? K::soft_kernel<true> : K::soft_kernel<false>;
+  // group vectors (2, or 4 with A / Bc), per-warp partials, argmax indices or
+  // TMEM slot, per-step weights (and gradients)
+  const size_t smem = sizeof(float) * ((size_t)(VJP ? 4 : 2) * K::J + 2 * 32 * 8 + (VJP ? 4 : 64) +
+                                       (size_t)(VJP ? 4 : 2) * sh.n);
+  if (smem > kMaxDynSmem) return BCJR_ERR_UNSUPPORTED;
+  int grid = 0;
+  int rc = grid_for(kern, K::NT, smem, sh.n_seq, &grid);
+  if (rc != BCJR_OK) return rc;
+  cap_grid_by_memory(&grid, sizeof(float) * (size_t)sh.n * K::J * (VJP ? 2 : 1) + sizeof(double) * sh.n +
+                                (VJP ? sizeof(float4) * K::G * 4 * K::NT + sizeof(double) * 2 * K::S : 0));
+  K::Params P{};
+  auto layout = [&](Arena& ar) {
+    P.cf = ar.take<float4>(K::CB4);
+    P.cb = ar.take<float4>(K::CB4);
+    P.hist_l = ar.take<float>((size_t)grid * sh.n * K::J);
+    P.hist_a = VJP ? ar.take<float>((size_t)grid * sh.n * K::J) : nullptr;
+    P.hist_c = ar.take<double>((size_t)grid * sh.n);
+    P.gc1 = VJP ? ar.take<float4>((size_t)grid * K::G * 4 * K::NT) : nullptr;
+    P.gc_part = VJP ? ar.take<double>((size_t)grid * 2 * K::S) : nullptr;
+  };
+  Arena sizing;
+  layout(sizing);
+  void* mem = nullptr;
+  if (int arc = scratch_alloc(&mem, sizing.off, st)) return arc;
+  Arena ar;
+  ar.base = static_cast<char*>(mem);
+  layout(ar);
+  P.w = a.w; P.gsoft = a.gsoft; P.gZ = a.gZ;
+  P.out_soft = a.out_soft; P.out_logZ = a.out_logZ; P.out_argmax = a.out_argmax; P.grad_w = a.grad_w;
+  P.n_seq = sh.n_seq; P.len = sh.len; P.n = sh.n;
+  P.sk = (float)std::sqrt(1.4426950408889634 / (double)a.T);
+  P.two_over_T = (float)(2.0 / (double)a.T);
+  K::make_codebooks<<<K::CB4 / 256, 256, 0, st>>>(a.c, P.sk, const_cast<float4*>(P.cf), const_cast<float4*>(P.cb));
+  kern<<<grid, K::NT, smem, st>>>(P);
+  if (VJP) K::reduce_gc<<<2 * K::S / 256, 256, 0, st>>>(P.gc_part, grid, a.grad_c);
+  cudaError_t le = cudaGetLastError();
+  cudaError_t fe = cudaFreeAsync(mem, st);
+  if (le != cudaSuccess || fe != cudaSuccess) return BCJR_ERR_CUDA;
+  return BCJR_OK;
+}
 
 template <int MODE>
 int run_sweep(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   constexpr bool VJP = MODE == bcjr::MODE_VJP;
   if (use_l16(sh)) return run_l16<MODE>(sh, a, st);
+  if (use_l16v2(sh)) return run_l16v2<MODE>(sh, a, st);
   SweepKernel kern = pick_sweep<MODE>(sh.V, sh.D);
   if (!kern) return BCJR_ERR_UNSUPPORTED;
   const int threads = threads_for(sh.J);

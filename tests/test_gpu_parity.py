@@ -175,6 +175,50 @@ def test_l16_block_kernel_matches_generic_kernel(monkeypatch):
     assert_grad(fast[2][rows], rv["grad_w"], "grad_w")
 
 
+def test_l16_vector_kernel_matches_generic_kernel(monkeypatch):
+    """The specialised L=16, k=2, V=2 kernels against the generic kernels on
+    300 sequences (more than one per CTA) of 48 steps (96 weights), T=0.05,
+    with gZ; then against the oracle on a few rows."""
+    w, c, g = I.random_case(16, 2, 2, 300, 96, seed=919)
+    gZ = torch.randn(300, generator=torch.Generator().manual_seed(7))
+    wd, cd, gd, gzd = w.to(DEV), c.to(DEV), g.to(DEV), gZ.to(DEV)
+    fast = [x.cpu().numpy() for x in lib.soft_codeword(wd, cd, 16, 2, 2, 0.05) + lib.vjp(wd, cd, 16, 2, 2, 0.05, gd, gzd)]
+    am_fast = lib.posterior_argmax(wd, cd, 16, 2, 2, 0.05).cpu().numpy()
+    assert lib.get_device_error() == 0
+    monkeypatch.setenv("BCJR_GENERIC_ONLY", "1")
+    gen = [x.cpu().numpy() for x in lib.soft_codeword(wd, cd, 16, 2, 2, 0.05) + lib.vjp(wd, cd, 16, 2, 2, 0.05, gd, gzd)]
+    am_gen = lib.posterior_argmax(wd, cd, 16, 2, 2, 0.05).cpu().numpy()
+    assert_soft(fast[0], gen[0], c)
+    assert_logZ(fast[1], gen[1], 16, 4, 48)
+    assert_grad(fast[2], gen[2], "grad_w")
+    assert_grad(fast[3], gen[3], "grad_c")
+    assert (am_fast == am_gen).mean() > 0.999
+    rows = [0, 147, 148, 299]
+    ref = oracle.soft(w[rows], c, 16, 2, 2, 0.05)
+    assert_logZ(fast[1][rows], ref["logZ"], 16, 4, 48)
+    assert_soft(fast[0][rows], ref["soft"], c)
+    rv = oracle.vjp(w[rows], c, 16, 2, 2, 0.05, g[rows], gZ[rows])
+    assert_grad(fast[2][rows], rv["grad_w"], "grad_w")
+    mask = unique_argmax_mask(ref["top2"])
+    np.testing.assert_array_equal(am_fast[rows][mask], ref["argmax"][mask])
+
+
+def test_l16_vector_kernel_longest(monkeypatch):
+    """V=2 at len = 8192 (4096 steps, the longest supported), biased upstream
+    gradient: specialised against generic kernels."""
+    w, c, g = I.random_case(16, 2, 2, 2, 8192, seed=929)
+    g[1] += 1.0
+    wd, cd, gd = w.to(DEV), c.to(DEV), g.to(DEV)
+    fast = [x.cpu().numpy() for x in lib.soft_codeword(wd, cd, 16, 2, 2, 0.1) + lib.vjp(wd, cd, 16, 2, 2, 0.1, gd)]
+    assert lib.get_device_error() == 0
+    monkeypatch.setenv("BCJR_GENERIC_ONLY", "1")
+    gen = [x.cpu().numpy() for x in lib.soft_codeword(wd, cd, 16, 2, 2, 0.1) + lib.vjp(wd, cd, 16, 2, 2, 0.1, gd)]
+    assert_soft(fast[0], gen[0], c)
+    assert_logZ(fast[1], gen[1], 16, 4, 4096)
+    assert_grad(fast[2], gen[2], "grad_w")
+    assert_grad(fast[3], gen[3], "grad_c")
+
+
 def test_l16_viterbi_matches_generic_and_oracle(monkeypatch):
     """The block-layout L=16 Viterbi against the generic kernel (bit-exact) on
     40 sequences of 96 steps, including exact ties from a coarse codebook."""
