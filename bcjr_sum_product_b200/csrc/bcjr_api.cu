@@ -244,7 +244,7 @@ int run_l16v2(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   if (!VJP) kern = a.out_argmax ? K::soft_kernel<true> : K::soft_kernel<false>;
   // group vectors (2, or 4 with A / Bc), per-warp partials, argmax indices or
   // TMEM slot, per-step weights (and gradients)
-  const size_t smem = sizeof(float) * ((size_t)(VJP ? 4 : 2) * K::J + 2 * 32 * 8 + (VJP ? 4 : 64) +
+  const size_t smem = sizeof(float) * ((size_t)(VJP ? 4 : 2) * K::J + 2 * 32 * 8 + (VJP ? 4 : 64 + 4) +
                                        (size_t)(VJP ? 4 : 2) * sh.n);
   if (smem > kMaxDynSmem) return BCJR_ERR_UNSUPPORTED;
   int grid = 0;
@@ -256,6 +256,8 @@ int run_l16v2(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   auto layout = [&](Arena& ar) {
     P.cf = ar.take<float4>(K::CB4);
     P.cb = ar.take<float4>(K::CB4);
+    P.cf1 = ar.take<float2>(K::CB4);
+    P.cb1 = ar.take<float2>(K::CB4);
     P.hist_l = ar.take<float>((size_t)grid * sh.n * K::J);
     P.hist_a = VJP ? ar.take<float>((size_t)grid * sh.n * K::J) : nullptr;
     P.hist_c = ar.take<double>((size_t)grid * sh.n);
@@ -274,7 +276,8 @@ int run_l16v2(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   P.n_seq = sh.n_seq; P.len = sh.len; P.n = sh.n;
   P.sk = (float)std::sqrt(1.4426950408889634 / (double)a.T);
   P.two_over_T = (float)(2.0 / (double)a.T);
-  K::make_codebooks<<<K::CB4 / 256, 256, 0, st>>>(a.c, P.sk, const_cast<float4*>(P.cf), const_cast<float4*>(P.cb));
+  K::make_codebooks<<<K::CB4 / 256, 256, 0, st>>>(a.c, P.sk, const_cast<float4*>(P.cf), const_cast<float4*>(P.cb),
+                                                  const_cast<float2*>(P.cf1), const_cast<float2*>(P.cb1));
   kern<<<grid, K::NT, smem, st>>>(P);
   if (VJP) K::reduce_gc<<<2 * K::S / 256, 256, 0, st>>>(P.gc_part, grid, a.grad_c);
   cudaError_t le = cudaGetLastError();

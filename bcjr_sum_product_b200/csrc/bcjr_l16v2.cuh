@@ -47,6 +47,8 @@ struct Params {
   const float* w;        // [n_seq][len], len = 2 n
   const float4* cf;      // forward-order scaled codebook, CB4 float4
   const float4* cb;      // backward-order scaled codebook, CB4 float4
+  const float2* cf1;     // component 1 of cf, CB4 float2 (streamed when component 0 is in TMEM)
+  const float2* cb1;     // component 1 of cb, CB4 float2
   const float* gsoft;    // [n_seq][len] (VJP)
   const float* gZ;       // [n_seq] or null (VJP)
   float* out_soft;       // [n_seq][len] or null
@@ -67,7 +69,7 @@ struct Params {
 // cb[(k * 8 + p) * 512 + tau]: backward group (h = 8e + k, mid), members lo = 2p, 2p + 1;
 // each float4 = (c0(first), c0(second), c1(first), c1(second)) * sk.
 __global__ void make_codebooks(const float* __restrict__ c, float sk, float4* __restrict__ cf,
-                               float4* __restrict__ cb) {
+                               float4* __restrict__ cb, float2* __restrict__ cf1, float2* __restrict__ cb1) {
   const int x = blockIdx.x * blockDim.x + threadIdx.x;
   if (x >= CB4) return;
   const int tau = x & (NT - 1), p = (x >> 9) & 7, k = x >> 12;
@@ -75,9 +77,11 @@ __global__ void make_codebooks(const float* __restrict__ c, float sk, float4* __
   const int lo = 8 * e + k;
   const int f0 = ((2 * p) << 12) | (mid << 4) | lo, f1 = ((2 * p + 1) << 12) | (mid << 4) | lo;
   cf[x] = make_float4(c[2 * f0] * sk, c[2 * f1] * sk, c[2 * f0 + 1] * sk, c[2 * f1 + 1] * sk);
+  cf1[x] = make_float2(c[2 * f0 + 1] * sk, c[2 * f1 + 1] * sk);
   const int h = 8 * e + k;
   const int b0 = (h << 12) | (mid << 4) | (2 * p), b1 = b0 + 1;
   cb[x] = make_float4(c[2 * b0] * sk, c[2 * b1] * sk, c[2 * b0 + 1] * sk, c[2 * b1 + 1] * sk);
+  cb1[x] = make_float2(c[2 * b0 + 1] * sk, c[2 * b1 + 1] * sk);
 }
 
 // grad_c[q][v] = sum over CTAs of gc_part[cta][q][v]
@@ -87,6 +91,23 @@ __global__ void reduce_gc(const double* __restrict__ part, int nparts, float* __
   double a = 0.0;
   for (int p = 0; p < nparts; ++p) a += part[(size_t)p * 2 * S + x];
   out[x] = (float)a;
+}
+
+// Component 0 of this thread's 8 groups x 8 member pairs of a codebook copy
+// into its 128 tensor-memory columns (column 16 k + 2 p + lane).
+__device__ __forceinline__ void stage_c0(const float4* __restrict__ cp, uint32_t tbase) {
+#pragma unroll
+  for (int k = 0; k < G; ++k) {
+    float v[16];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      const float4 cw = __ldg(cp + (k * 8 + p) * NT);
+      v[2 * p] = cw.x;
+      v[2 * p + 1] = cw.y;
+    }
+    l16::tmem_st16(tbase + 16 * k, v);
+  }
+  l16::tmem_wait_st();
 }
 
 __device__ __forceinline__ float pick8(const float (&v)[16], int e, int i) { return e ? v[8 + i] : v[i]; }
@@ -111,18 +132,28 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
   float* lb[2] = {smem, smem + J};                     // negated group vectors (ping-pong)
   float* rec = smem + 2 * J;                           // [2][32][8] per-warp partials
   int* arec = reinterpret_cast<int*>(rec + 2 * 32 * 8);  // [2][32] argmax index
-  float* wsc = reinterpret_cast<float*>(arec + 64);    // [n][2]: -w'
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(arec + 64);  // [4]
+  float* wsc = reinterpret_cast<float*>(tslot + 4);    // [n][2]: -w'
 
   float* hist = P.hist_l + (size_t)blockIdx.x * n * J;
   double* hist_c = P.hist_c + (size_t)blockIdx.x * n;
-  const float4* __restrict__ cf = P.cf + tid;
-  const float4* __restrict__ cb = P.cb + tid;
+  const float2* __restrict__ cf1 = P.cf1 + tid;
+  const float2* __restrict__ cb1 = P.cb1 + tid;
   const float2 neg1 = f2s(-1.f);
   const int hoff = mid * 16 + 8 * e;                   // this thread's 8 entries of a history step
+
+  // tensor memory: component 0 of the codewords of the thread's groups of the
+  // current direction (128 columns), component 1 streams from L2
+  if (warp == 0) l16::tmem_alloc512(tslot);
+  l16::tmem_fence_before();
+  __syncthreads();
+  l16::tmem_fence_after();
+  const uint32_t tbase = tslot[0] + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(128 * (warp >> 2));
 
   for (int64_t seq = blockIdx.x; seq < P.n_seq; seq += gridDim.x) {
     const float* wq = P.w + seq * P.len;
     for (int x = tid; x < 2 * n; x += NT) wsc[x] = -wq[x] * P.sk;
+    stage_c0(P.cf + tid, tbase);
     __syncthreads();
 
     // ------------------------------------------------------------ forward
@@ -149,10 +180,12 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
 #pragma unroll
       for (int k = 0; k < G; ++k) {
         float2 x[8];
+        float c0v[16];
+        l16::tmem_ld16(tbase + 16 * k, c0v);
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
-          const float4 cw = __ldg(cf + (k * 8 + p) * NT);
-          const float2 d0 = __fadd2_rn(f2(cw.x, cw.y), nw0), d1 = __fadd2_rn(f2(cw.z, cw.w), nw1);
+          const float2 c1 = __ldg(cf1 + (k * 8 + p) * NT);
+          const float2 d0 = __fadd2_rn(f2(c0v[2 * p], c0v[2 * p + 1]), nw0), d1 = __fadd2_rn(c1, nw1);
           x[p] = __ffma2_rn(d1, d1, __ffma2_rn(d0, d0, f2(np[2 * p], np[2 * p + 1])));
         }
         const float m = min16(x);
@@ -189,6 +222,7 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
     }
 
     // ------------------------------------------------------------ backward
+    stage_c0(P.cb + tid, tbase);
     float Rrn = 0.f;
     double Cr = 0.0;
     float4 hsa = make_float4(0.f, 0.f, 0.f, 0.f), hsb = hsa;
@@ -229,11 +263,12 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
 #pragma unroll
       for (int k = 0; k < G; ++k) {            // group (h = 8e + k, mid), members lo
         float2 y[8], c0[8], c1[8];
+        float c0v[16];
+        l16::tmem_ld16(tbase + 16 * k, c0v);
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
-          const float4 cw = __ldg(cb + (k * 8 + p) * NT);
-          c0[p] = f2(cw.x, cw.y);
-          c1[p] = f2(cw.z, cw.w);
+          c0[p] = f2(c0v[2 * p], c0v[2 * p + 1]);
+          c1[p] = __ldg(cb1 + (k * 8 + p) * NT);
           const float2 d0 = __fadd2_rn(c0[p], nw0), d1 = __fadd2_rn(c1[p], nw1);
           y[p] = __ffma2_rn(d1, d1, __ffma2_rn(d0, d0, f2(nr[2 * p], nr[2 * p + 1])));
         }
@@ -301,6 +336,11 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
     }
     __syncthreads();
   }
+
+  l16::tmem_fence_before();
+  __syncthreads();
+  l16::tmem_fence_after();
+  if (warp == 0) l16::tmem_dealloc512(tslot[0]);
 }
 
 // ------------------------------------------------------------ VJP
@@ -332,7 +372,7 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
   double* hist_c = P.hist_c + (size_t)blockIdx.x * n;
   float4* gc1 = P.gc1 + (size_t)blockIdx.x * (G * 4 * NT) + tid;
   double* gcp = P.gc_part + (size_t)blockIdx.x * 2 * S;
-  const float4* __restrict__ cf = P.cf + tid;
+  const float2* __restrict__ cf1 = P.cf1 + tid;
   const float4* __restrict__ cb = P.cb + tid;
   const float2 neg1 = f2s(-1.f);
   const int hoff = mid * 16 + 8 * e;
@@ -350,6 +390,7 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
     const float* wq = P.w + seq * P.len;
     const float* gq = P.gsoft + seq * P.len;
     for (int x = tid; x < 2 * n; x += NT) { wsc[x] = -wq[x] * P.sk; gsc[x] = gq[x] / P.sk; }
+    stage_c0(P.cf + tid, tbase);   // the forward's component 0 (the backward's gradient later)
     __syncthreads();
 
     // ------------------------------------------------------------ forward
@@ -385,10 +426,11 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
 #pragma unroll 1
       for (int k = 0; k < G; ++k) {
         float2 x[8], z[8];
+        float c0v[16];
+        l16::tmem_ld16(tbase + 16 * k, c0v);
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
-          const float4 cw = __ldg(cf + (k * 8 + p) * NT);
-          const float2 c0 = f2(cw.x, cw.y), c1 = f2(cw.z, cw.w);
+          const float2 c0 = f2(c0v[2 * p], c0v[2 * p + 1]), c1 = __ldg(cf1 + (k * 8 + p) * NT);
           const float2 d0 = __fadd2_rn(c0, nw0), d1 = __fadd2_rn(c1, nw1);
           x[p] = __ffma2_rn(d1, d1, __ffma2_rn(d0, d0, f2(np[2 * p], np[2 * p + 1])));
           z[p] = __ffma2_rn(g1, c1, __ffma2_rn(g0, c0, f2(ap[2 * p], ap[2 * p + 1])));
