@@ -54,10 +54,12 @@ LEDGERS = {
     (2, 2): {"soft": {"fp32": 4.94 + 8.94, "mufu": 2.0}, "vjp": {"fp32": 10.88 + 22.69, "mufu": 2.0}},
 }
 LEDGER = LEDGERS[(2, 1)]
-# DRAM bytes per sequence (read + write) of each L=16 sweep kernel, from one
+# DRAM bytes per sequence (read + write) of each L=16, V=1 sweep kernel, from one
 # ncu capture of 16 qtip sequences (profiles/vjp_kernel_qtip16.md,
 # profiles/soft_kernel_qtip16.md); set to None whenever the kernel changes.
-TRAFFIC_PER_SEQ = {"vjp": 1002.29e6 / 16, "soft": 445.70e6 / 16}
+# (A 16-sequence capture of the V=2 kernels keeps their histories in L2, so it
+# does not scale to a full launch; their traffic is reported as null.)
+TRAFFIC_PER_SEQ = {"vjp": 1003.29e6 / 16, "soft": 448.17e6 / 16}
 FP32_PER_CLK_SM = 128.0   # FFMA lanes per SM per clock (measured 123.5 FFMA, 126 FFMA2 on this machine)
 MUFU_PER_CLK_SM = 16.0    # ex2 per SM per clock (measured 15.99 on this machine)
 N_SM = 148
@@ -343,8 +345,12 @@ def main():
     ms_dom = ms_vjp if dominant == "vjp" else ms_soft
     achieved = units / (ms_dom / 1e3)
     block_layout = (L, k, V) == (16, 2, 1)
-    kernel = (f"bcjr::l16::{dominant}_kernel" if block_layout else
-              f"bcjr::bcjr_sweep_kernel<{V},{k * V},{1 if dominant == 'vjp' else 0}>")
+    if block_layout:
+        kernel = f"bcjr::l16::{dominant}_kernel"
+    elif (L, k, V) == (16, 2, 2):
+        kernel = f"bcjr::l16v2::{dominant}_kernel"
+    else:
+        kernel = f"bcjr::bcjr_sweep_kernel<{V},{k * V},{1 if dominant == 'vjp' else 0}>"
     roofline = None
     if ledger is not None:
         peak = peak_units_per_s(dominant, fmax, ledger)
