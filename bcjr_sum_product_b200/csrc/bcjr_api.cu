@@ -1,5 +1,6 @@
 // Host side of the C ABI declared in include/bcjr.h: argument validation,
 // stream-ordered scratch allocation, kernel selection and launch.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -492,6 +493,45 @@ int viterbi_decode(const float* w, int64_t n_seq, int64_t len, int L, int k, int
       (rc = check_dev_ptr(out_cost, true)))
     return rc;
   return run_viterbi(sh, w, codebook, out_states, out_cost, static_cast<cudaStream_t>(stream));
+}
+
+int bcjr_qat_step(float* w, const float* w_target, int64_t n_seq, int64_t len, int L, int k, int V, float* codebook,
+                  float T, float lr_w, float lr_c, float* out_soft, float* out_loss, float* grad_w,
+                  float* grad_codebook, void* stream) {
+  Shape sh;
+  int rc = check_shape(n_seq, len, L, k, V, &sh);
+  if (rc) return rc;
+  if ((rc = check_T(T))) return rc;
+  if (!std::isfinite(lr_w) || !std::isfinite(lr_c)) return BCJR_ERR_INVALID_ARG;
+  if ((rc = check_dev_ptr(codebook, false)) || (rc = check_dev_ptr(grad_codebook, false))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (n_seq == 0) {
+    return cudaMemsetAsync(grad_codebook, 0, sizeof(float) * (size_t)sh.S * sh.V, st) == cudaSuccess
+               ? BCJR_OK
+               : BCJR_ERR_CUDA;
+  }
+  if ((rc = check_dev_ptr(w, false)) || (rc = check_dev_ptr(w_target, false)) ||
+      (rc = check_dev_ptr(out_soft, false)) || (rc = check_dev_ptr(out_loss, true)) ||
+      (rc = check_dev_ptr(grad_w, false)))
+    return rc;
+  SweepArgs a{w, codebook, T, nullptr, nullptr, out_soft, nullptr, nullptr, nullptr, nullptr};
+  if ((rc = run_sweep<bcjr::MODE_SOFT>(sh, a, st))) return rc;
+  const int64_t nw = n_seq * len;
+  void* g = nullptr;
+  if ((rc = scratch_alloc(&g, sizeof(float) * (size_t)nw, st))) return rc;
+  bcjr::recon_grad_kernel<<<(unsigned)std::min<int64_t>(n_seq, 148 * 64), 256, 0, st>>>(
+      out_soft, w_target, n_seq, len, static_cast<float*>(g), out_loss);
+  SweepArgs b{w, codebook, T, static_cast<float*>(g), nullptr, nullptr, nullptr, nullptr, grad_w, grad_codebook};
+  rc = run_sweep<bcjr::MODE_VJP>(sh, b, st);
+  if (rc == BCJR_OK) {
+    const int64_t sv = (int64_t)sh.S * sh.V;
+    bcjr::sgd_kernel<<<(unsigned)std::min<int64_t>((nw + 255) / 256, 148 * 16), 256, 0, st>>>(w, grad_w, lr_w, nw);
+    if (lr_c != 0.f)
+      bcjr::sgd_kernel<<<(unsigned)((sv + 255) / 256), 256, 0, st>>>(codebook, grad_codebook, lr_c, sv);
+    if (cudaGetLastError() != cudaSuccess) rc = BCJR_ERR_CUDA;
+  }
+  if (cudaFreeAsync(g, st) != cudaSuccess && rc == BCJR_OK) rc = BCJR_ERR_CUDA;
+  return rc;
 }
 
 int bcjr_get_device_error(void* stream) {

@@ -443,6 +443,40 @@ __global__ void reduce_gc_kernel(const double* __restrict__ part, int nparts, in
   out[x] = (float)a;
 }
 
+// Self-reconstruction loss of a sequence and its upstream gradient:
+// g = 2 (w_hat - w_target), loss[q] = sum (w_hat - w_target)^2; blocks of 256
+// threads stride over the sequences, each reduced in a fixed order.
+__global__ void recon_grad_kernel(const float* __restrict__ soft, const float* __restrict__ target, int64_t n_seq,
+                                  int64_t len, float* __restrict__ g, float* __restrict__ loss) {
+  __shared__ float part[8];
+  for (int64_t q = blockIdx.x; q < n_seq; q += gridDim.x) {
+    const float* a = soft + q * len;
+    const float* b = target + q * len;
+    float* gq = g + q * len;
+    float acc = 0.f;
+    for (int64_t x = threadIdx.x; x < len; x += blockDim.x) {
+      const float d = a[x] - b[x];
+      gq[x] = 2.f * d;
+      acc = fmaf(d, d, acc);
+    }
+    acc = warp_sum(acc);
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0 && loss) {
+      float tot = 0.f;
+      for (int i = 0; i < (int)(blockDim.x >> 5); ++i) tot += part[i];
+      loss[q] = tot;
+    }
+    __syncthreads();
+  }
+}
+
+// x <- x - lr * g
+__global__ void sgd_kernel(float* __restrict__ x, const float* __restrict__ g, float lr, int64_t n) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    x[i] = fmaf(-lr, g[i], x[i]);
+}
+
 // c'(s) = sk * c(s)
 __global__ void scale_codebook_kernel(const float* __restrict__ c, int SV, float sk, float* __restrict__ cs) {
   int x = blockIdx.x * blockDim.x + threadIdx.x;

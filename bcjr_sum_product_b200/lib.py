@@ -52,6 +52,7 @@ def load(path: str = LIB_PATH):
             lib.bcjr_vjp.argtypes = [P, i64, i64, i32, i32, i32, P, f32, P, P, P, P, P]
             lib.viterbi_decode.argtypes = [P, i64, i64, i32, i32, i32, P, P, P, P]
             lib.bcjr_posterior_argmax.argtypes = [P, i64, i64, i32, i32, i32, P, f32, P, P]
+            lib.bcjr_qat_step.argtypes = [P, P, i64, i64, i32, i32, i32, P, f32, f32, f32, P, P, P, P, P]
             lib.bcjr_get_device_error.argtypes = [P]
             lib.bcjr_strerror.argtypes = [i32]
             lib.bcjr_strerror.restype = ctypes.c_char_p
@@ -129,6 +130,33 @@ def vjp(w: torch.Tensor, codebook: torch.Tensor, L: int, k: int, V: int, T: floa
                          _ptr(grad_logZ), _ptr(grad_w), _ptr(grad_codebook), _stream(stream))
     _check(rc, "bcjr_vjp")
     return grad_w, grad_codebook
+
+
+def qat_step(w: torch.Tensor, w_target: torch.Tensor, codebook: torch.Tensor, L: int, k: int, V: int, T: float,
+             lr_w: float, lr_c: float = 0.0, out_soft: Optional[torch.Tensor] = None,
+             out_loss: Optional[torch.Tensor] = None, grad_w: Optional[torch.Tensor] = None,
+             grad_codebook: Optional[torch.Tensor] = None,
+             stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor]:
+    """bcjr_qat_step: one self-reconstruction QAT step; updates ``w`` (and the
+    codebook when ``lr_c`` != 0) in place and returns (w_hat, loss per sequence,
+    dl/dw, dl/dcodebook), all taken before the update."""
+    _dev(w, "w"); _dev(w_target, "w_target"); _dev(codebook, "codebook")
+    n_seq, seq_len = w.shape
+    if tuple(w_target.shape) != (n_seq, seq_len):
+        raise ValueError("w_target must have the shape of w")
+    if out_soft is None:
+        out_soft = torch.empty_like(w)
+    if out_loss is None:
+        out_loss = torch.empty(n_seq, device=w.device, dtype=torch.float32)
+    if grad_w is None:
+        grad_w = torch.empty_like(w)
+    if grad_codebook is None:
+        grad_codebook = torch.empty_like(codebook)
+    rc = load().bcjr_qat_step(_ptr(w), _ptr(w_target), n_seq, seq_len, L, k, V, _ptr(codebook), float(T),
+                              float(lr_w), float(lr_c), _ptr(out_soft), _ptr(out_loss), _ptr(grad_w),
+                              _ptr(grad_codebook), _stream(stream))
+    _check(rc, "bcjr_qat_step")
+    return out_soft, out_loss, grad_w, grad_codebook
 
 
 def viterbi_decode(w: torch.Tensor, codebook: torch.Tensor, L: int, k: int, V: int,

@@ -11,12 +11,14 @@ seed 2).  Metric: state-updates/s = n_seq * n_steps * 2^L per step / time
 (weights/s reported alongside).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload qtip|mid|mlp|layer|tiny] [--temp T]
+                    [--workload qtip|mid|mlp|layer|tiny] [--temp T] [--qat]
 
 The default workload is the QTIP-scale one above.  ``--workload`` measures the
 other seeded workloads of the inputs module with the same timing rules (``mid``
 is forward only: soft codeword and logZ; ``mlp`` takes ``--temp`` from
-{1, 0.1, 0.01}).
+{1, 0.1, 0.01}).  ``--qat`` times one self-reconstruction QAT step per
+iteration instead (``bcjr_qat_step``: soft codeword, loss and its upstream
+gradient, VJP and the in-place SGD update of the weights, lr 1e-3).
 
 N > 1 runs under torch.distributed.run, one rank per GPU, each rank on its own
 copy of the workload (weak scaling); the codebook gradient is summed across
@@ -145,6 +147,10 @@ def cpu_baseline(wl, inp, n_rows: int, T: float, do_vjp: bool):
                       f"fp64 C oracle with OpenMP over sequences; {dt:.1f} s"}
 
 
+def units_e2e(wl, n_seq: int) -> int:
+    return n_seq * wl.n_steps * wl.S
+
+
 def describe(wl, T: float, do_vjp: bool) -> str:
     mats = ", ".join(f"{r}x{c}" for r, c in wl.matrices)
     what = "soft codeword + logZ + VJP" if do_vjp else "soft codeword + logZ"
@@ -212,6 +218,7 @@ def main():
                     help="profiling only: run on the first N sequences of the workload (not a bench number)")
     ap.add_argument("--workload", default=WORKLOAD, choices=["qtip", "mid", "mlp", "layer", "tiny"])
     ap.add_argument("--temp", type=float, default=None, help="temperature (one of the workload's)")
+    ap.add_argument("--qat", action="store_true", help="time bcjr_qat_step (self-reconstruction QAT step)")
     args = ap.parse_args()
     from bcjr_sum_product_b200 import inputs as I
     if args.temp is not None and args.temp not in I.WORKLOADS[args.workload].temps:
@@ -237,7 +244,7 @@ def main():
     lib.load()
 
     wl = I.WORKLOADS[args.workload]
-    do_vjp = "vjp" in wl.calls
+    do_vjp = "vjp" in wl.calls or args.qat
     inp = I.make(args.workload, rows=list(range(args.seqs)) if args.seqs > 0 else None, with_grad=do_vjp)
     T = args.temp if args.temp is not None else wl.temps[0]
     L, k, V = wl.L, wl.k, wl.V
@@ -252,7 +259,20 @@ def main():
     def local_vjp(wl_, cb_, g_):
         return lib.vjp(wl_, cb_, L, k, V, T, g_, grad_w=gw, grad_codebook=gc, stream=stream)
 
+    if args.qat:
+        if world > 1:
+            raise SystemExit("--qat runs on one GPU")
+        w_target = w.clone()
+        qloss = torch.empty(n_seq, device=dev)
+
+    def qat_step():
+        lib.qat_step(w, w_target, c, L, k, V, T, 1e-3, 0.0, out_soft=soft, out_loss=qloss, grad_w=gw,
+                     grad_codebook=gc, stream=stream)
+
     def step():
+        if args.qat:
+            qat_step()
+            return
         lib.soft_codeword(w, c, L, k, V, T, out_soft=soft, out_logZ=logZ, stream=stream)
         # each rank: VJP of its own sequences, then the codebook gradient summed over ranks
         if do_vjp:
@@ -275,10 +295,14 @@ def main():
         flush.fill_(1.0)  # L2 flush between timed iterations (outside the events)
         e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
         e0.record(stream)
-        lib.soft_codeword(w, c, L, k, V, T, out_soft=soft, out_logZ=logZ, stream=stream)
-        e1.record(stream)
-        if do_vjp:
-            bdist.vjp_data_parallel(local_vjp, w, c, g)
+        if args.qat:
+            qat_step()
+            e1.record(stream)
+        else:
+            lib.soft_codeword(w, c, L, k, V, T, out_soft=soft, out_logZ=logZ, stream=stream)
+            e1.record(stream)
+            if do_vjp:
+                bdist.vjp_data_parallel(local_vjp, w, c, g)
         e2.record(stream)
         e2.synchronize()
         soft_ms.append(e0.elapsed_time(e1)); vjp_ms.append(e1.elapsed_time(e2)); step_ms.append(e0.elapsed_time(e2))
@@ -300,7 +324,25 @@ def main():
 
     # e2e: through the public API with host buffers, copies inside the timed region
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and args.qat:
+        hw = inp.w.pin_memory(); hc = inp.c.pin_memory()
+        out_w_h = torch.empty_like(hw).pin_memory(); out_loss_h = torch.empty(n_seq).pin_memory()
+        h2d = 2 * hw.numel() * 4 + hc.numel() * 4
+        d2h = out_w_h.numel() * 4 + out_loss_h.numel() * 4
+        times = []
+        for _ in range(max(1, min(args.steps, 3))):
+            flush.fill_(1.0)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            w.copy_(hw, non_blocking=True); w_target.copy_(hw, non_blocking=True); c.copy_(hc, non_blocking=True)
+            qat_step()
+            out_w_h.copy_(w, non_blocking=True); out_loss_h.copy_(qloss, non_blocking=True)
+            b.record(stream)
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+        e2e = {"value": units_e2e(wl, n_seq) / (sum(times) / len(times) / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": sum(times) / len(times)}
+    elif not args.no_e2e:
         hw = inp.w.pin_memory(); hc = inp.c.pin_memory(); hg = inp.g.pin_memory() if do_vjp else None
         out_soft_h = torch.empty_like(hw).pin_memory(); out_logZ_h = torch.empty(n_seq).pin_memory()
         out_gw_h = torch.empty_like(hw).pin_memory() if do_vjp else None
@@ -342,10 +384,14 @@ def main():
     peaks, basis = measured_peaks()
     fmax = float(peaks.get("sm_max_mhz", 1965.0))
     dominant = "vjp" if do_vjp and ms_vjp >= ms_soft else "soft"
-    ms_dom = ms_vjp if dominant == "vjp" else ms_soft
+    if args.qat:
+        dominant = "step"
+    ms_dom = ms_step if args.qat else (ms_vjp if dominant == "vjp" else ms_soft)
     achieved = units / (ms_dom / 1e3)
     block_layout = (L, k, V) == (16, 2, 1)
-    if block_layout:
+    if args.qat:
+        kernel = "bcjr_qat_step (soft codeword + loss + VJP + update, all launches)"
+    elif block_layout:
         kernel = f"bcjr::l16::{dominant}_kernel"
     elif (L, k, V) == (16, 2, 2):
         kernel = f"bcjr::l16v2::{dominant}_kernel"
@@ -354,12 +400,14 @@ def main():
     roofline = None
     if ledger is not None:
         peak = peak_units_per_s(dominant, fmax, ledger)
-        tps = TRAFFIC_PER_SEQ.get(dominant) if block_layout else None
+        tps = TRAFFIC_PER_SEQ.get(dominant) if block_layout and not args.qat else None
         roofline = {"bound": "alu", "kernel": kernel, "achieved": achieved, "peak": peak,
                     "unit": UNIT, "frac": achieved / peak, "traffic": (tps * n_seq) if tps else None,
                     "traffic_note": "DRAM bytes per launch, scaled from an ncu capture of 16 sequences",
-                    "peak_basis": f"{N_SM} SMs x min(128 FP32 / {ledger[dominant]['fp32']}, 16 MUFU / "
-                                  f"{ledger[dominant]['mufu']}) units/clk at sm_max {fmax:.0f} MHz ({basis})"}
+                    "peak_basis": (f"{N_SM} SMs x min(128 FP32 / {ledger[dominant]['fp32']}, 16 MUFU / "
+                                   f"{ledger[dominant]['mufu']}) units/clk at sm_max {fmax:.0f} MHz ({basis})"
+                                   if dominant != "step" else
+                                   f"{N_SM} SMs, soft + VJP ledger, at sm_max {fmax:.0f} MHz ({basis})")}
         if do_vjp:
             roofline["step_frac"] = value / world / peak_units_per_s("step", fmax, ledger)
         if clocks.get("sm_mhz"):
@@ -374,7 +422,10 @@ def main():
         cores = os.cpu_count() or 1
         cpu = cpu_baseline(wl, inp, max(1, min(cores, 16, n_seq)), T, do_vjp)
 
-    line = {"metric": metric_for(wl, do_vjp), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+    metric = metric_for(wl, do_vjp)
+    if args.qat:
+        metric = f"BCJR-QAT self-reconstruction step (soft + loss + VJP + update): state-updates/s on the {wl.name} workload, 1 B200"
+    line = {"metric": metric, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": describe(wl, T, do_vjp),
@@ -382,9 +433,9 @@ def main():
                        "l2": "flushed between timed iterations (256 MB write outside the events)",
                        "parallelism": f"dp{world}" if world > 1 else "single"},
             "weights_per_s": world * n_seq * wl.seq_len / (ms_step / 1e3),
-            "ms_soft": ms_soft, "ms_vjp": ms_vjp, "wall_s": wall,
+            "ms_soft": None if args.qat else ms_soft, "ms_vjp": None if args.qat else ms_vjp, "wall_s": wall,
             "ms_step_min_max": [min(step_ms), max(step_ms)],
-            "gpu_launches": (5 if do_vjp else 2) * args.steps,
+            "gpu_launches": (7 if args.qat else 5 if do_vjp else 2) * args.steps,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks}
     if line_note:
         line["note"] = line_note

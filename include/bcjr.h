@@ -157,6 +157,33 @@ BCJR_API int bcjr_soft_codeword_noalloc(const float* w, int64_t n_seq, int64_t l
                                         void* stream);
 
 /*
+ * One step of quantisation-aware training by self-reconstruction (BCJR-QAT,
+ * Technical Summary "Core Mechanism": the soft codeword of the latent weights
+ * stands in for the quantised weights, and T is annealed from T0 towards a
+ * near-zero T_end over the steps, one call per step with its own T).  With
+ * w_hat the soft codeword of w at temperature T,
+ *   loss[q] = sum_{t,v} (w_hat[q][t*V+v] - w_target[q][t*V+v])^2,
+ * the call computes w_hat and the loss, the VJP of sum_q loss[q] (upstream
+ * gradient 2 (w_hat - w_target), no gradient on logZ), and then updates in place
+ *   w        <- w        - lr_w * dl/dw
+ *   codebook <- codebook - lr_c * dl/dc      (only when lr_c != 0)
+ *   w             [n_seq][len]  latent weights (input; updated in place)
+ *   w_target      [n_seq][len]  target weights (input)
+ *   codebook      [2^L][V]      codewords (input; updated in place when lr_c != 0)
+ *   out_soft      [n_seq][len]  w_hat before the update (output)
+ *   out_loss      [n_seq]       loss per sequence before the update (output, may be NULL)
+ *   grad_w        [n_seq][len]  dl/dw (output)
+ *   grad_codebook [2^L][V]      dl/dc (output)
+ * All device pointers; w, w_target, out_soft and grad_w must not overlap.
+ * lr_w and lr_c must be finite (BCJR_ERR_INVALID_ARG otherwise).  Every step
+ * runs in the library's kernels on `stream`; the upstream gradient lives in
+ * library scratch.
+ */
+BCJR_API int bcjr_qat_step(float* w, const float* w_target, int64_t n_seq, int64_t len, int L, int k, int V,
+                           float* codebook, float T, float lr_w, float lr_c, float* out_soft, float* out_loss,
+                           float* grad_w, float* grad_codebook, void* stream);
+
+/*
  * Synchronises `stream` and returns BCJR_OK, or BCJR_ERR_CUDA if the stream
  * holds a CUDA error, or the first device-side error recorded by a kernel of
  * this library since the last call (BCJR_ERR_TIMEOUT for a bounded wait that

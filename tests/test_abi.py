@@ -69,6 +69,12 @@ def test_shape_and_temperature_validation_without_gpu():
     assert L.viterbi_decode(None, 1, 8, 17, 2, 1, None, None, None, None) == lib.BCJR_ERR_UNSUPPORTED
     assert L.bcjr_vjp(None, 1, 8, 8, 2, 1, None, 0.5, None, None, None, None, None) == lib.BCJR_ERR_INVALID_ARG
     assert L.bcjr_posterior_argmax(None, 1, 8, 8, 2, 1, None, -2.0, None, None) == lib.BCJR_ERR_INVALID_ARG
+    qat = L.bcjr_qat_step
+    assert qat(None, None, 1, 8, 17, 2, 1, None, 0.5, 1e-3, 0.0, None, None, None, None, None) == lib.BCJR_ERR_UNSUPPORTED
+    assert qat(None, None, 1, 8, 8, 2, 1, None, 0.0, 1e-3, 0.0, None, None, None, None, None) == lib.BCJR_ERR_INVALID_ARG
+    assert qat(None, None, 1, 8, 8, 2, 1, None, 0.5, float("nan"), 0.0, None, None, None, None, None) == lib.BCJR_ERR_INVALID_ARG
+    assert qat(None, None, 1, 8, 8, 2, 1, None, 0.5, 1e-3, float("inf"), None, None, None, None, None) == lib.BCJR_ERR_INVALID_ARG
+    assert qat(None, None, 1, 8, 8, 2, 1, None, 0.5, 1e-3, 0.0, None, None, None, None, None) == lib.BCJR_ERR_INVALID_ARG
 
 
 def test_binding_rejects_host_tensors():
