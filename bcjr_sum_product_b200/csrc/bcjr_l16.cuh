@@ -343,27 +343,25 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
             const float2 d = __fadd2_rn(f2(cb[bidx(2 * g, lo)], cb[bidx(2 * g + 1, lo)]), nw2);
             y[lo] = __ffma2_rn(d, d, f2s(nr[lo]));
           }
-          const float2 m = f2(fminf(fminf(y[0].x, y[1].x), fminf(y[2].x, y[3].x)),
-                              fminf(fminf(y[0].y, y[1].y), fminf(y[2].y, y[3].y)));
-          // posterior factor of each group: 2^(K - m' - n_sigma)
-          const float2 ge = __fadd2_rn(__fadd2_rn(f2s(K), f2(-hs[2 * g], -hs[2 * g + 1])), __fmul2_rn(m, neg1));
-          const float2 gf = f2(ex2f(ge.x), ex2f(ge.y));
+          // the posterior directly, p = 2^(K - n_sigma - y'), one ex2 per state
+          const float2 kh = __fadd2_rn(f2s(K), f2(-hs[2 * g], -hs[2 * g + 1]));
           float2 ssum = f2s(0.f);
 #pragma unroll
           for (int lo = 0; lo < 4; ++lo) {
-            const float2 a = __ffma2_rn(y[lo], neg1, m);
-            const float2 u = f2(ex2f(a.x), ex2f(a.y));
-            ssum = __fadd2_rn(ssum, u);
-            const float2 pp = __fmul2_rn(u, gf);
+            const float2 a = __ffma2_rn(y[lo], neg1, kh);
+            const float2 pp = f2(ex2f(a.x), ex2f(a.y));
+            ssum = __fadd2_rn(ssum, pp);
             accc = __ffma2_rn(pp, f2(cb[bidx(2 * g, lo)], cb[bidx(2 * g + 1, lo)]), accc);
-            accp = __fadd2_rn(accp, pp);
             if constexpr (ARGMAX) {
               arg_better(bestp, bestq, pp.x, ((2 * g) << 14) | (mid << 2) | lo);
               arg_better(bestp, bestq, pp.y, ((2 * g + 1) << 14) | (mid << 2) | lo);
             }
           }
-          nout[2 * g] = (m.x - Rrn) - lg2f(ssum.x);
-          nout[2 * g + 1] = (m.y - Rrn) - lg2f(ssum.y);
+          accp = __fadd2_rn(accp, ssum);
+          // negated log rho_{t-1} = (K - n_sigma) - lg2 sum p (+inf, i.e. rho = 0, when the
+          // group's posterior mass underflows; it then moves no posterior by more than that mass)
+          nout[2 * g] = (kh.x - Rrn) - lg2f(ssum.x);
+          nout[2 * g + 1] = (kh.y - Rrn) - lg2f(ssum.y);
         }
         if (t >= 1) {
 #pragma unroll
@@ -649,20 +647,17 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
             const float2 dd = __fadd2_rn(c2[lo], nw2);
             y[lo] = __ffma2_rn(dd, dd, f2s(nr[lo]));
           }
-          const float2 m = f2(fminf(fminf(y[0].x, y[1].x), fminf(y[2].x, y[3].x)),
-                              fminf(fminf(y[0].y, y[1].y), fminf(y[2].y, y[3].y)));
-          const float2 ge = __fadd2_rn(__fadd2_rn(f2s(K), f2(-hs0, -hs1)), __fmul2_rn(m, neg1));
-          const float2 gf = f2(ex2f(ge.x), ex2f(ge.y));
+          // the posterior directly, p = 2^(K - n_sigma - y'), one ex2 per state
+          const float2 kh = __fadd2_rn(f2s(K), f2(-hs0, -hs1));
           const float2 ah = f2(ha0 - hbt, ha1 - hbt);   // A - K + gZ
           float2 ssum = f2s(0.f), num = f2s(0.f);
 #pragma unroll
           for (int lo = 0; lo < 4; ++lo) {
-            const float2 a = __ffma2_rn(y[lo], neg1, m);
-            const float2 u = f2(ex2f(a.x), ex2f(a.y));
-            ssum = __fadd2_rn(ssum, u);
+            const float2 a = __ffma2_rn(y[lo], neg1, kh);
+            const float2 pp = f2(ex2f(a.x), ex2f(a.y));
+            ssum = __fadd2_rn(ssum, pp);
             const float2 z = __ffma2_rn(g2, c2[lo], f2s(bc[lo]));          // Bc + h
-            num = __ffma2_rn(u, z, num);
-            const float2 pp = __fmul2_rn(u, gf);
+            num = __ffma2_rn(pp, z, num);
             const float2 G = __fmul2_rn(pp, __fadd2_rn(z, ah));
             accG = __fadd2_rn(accG, G);
             accGc = __ffma2_rn(G, c2[lo], accGc);
@@ -673,12 +668,14 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
             gcb[2 * lo + 1] = gc.y;
           }
           tmem_st8(tbase + 16 * k + 8 * g, gcb);
-          nout[2 * g] = (m.x - Rrn) - lg2f(ssum.x);
-          nout[2 * g + 1] = (m.y - Rrn) - lg2f(ssum.y);
-          bout[2 * g] = __fdividef(num.x, ssum.x);
-          bout[2 * g + 1] = __fdividef(num.y, ssum.y);
+          // negated log rho_{t-1} = (K - n_sigma) - lg2 sum p; a group whose posterior mass
+          // underflows gets rho = 0 (+inf) and Bc = 0, moving no posterior by more than that mass
+          nout[2 * g] = (kh.x - Rrn) - lg2f(ssum.x);
+          nout[2 * g + 1] = (kh.y - Rrn) - lg2f(ssum.y);
+          bout[2 * g] = (ssum.x > 0.f) ? __fdividef(num.x, ssum.x) : 0.f;
+          bout[2 * g + 1] = (ssum.y > 0.f) ? __fdividef(num.y, ssum.y) : 0.f;
           // posterior of the two step t-1 groups, P(i) = sum_lo p
-          const float2 pg = __fmul2_rn(gf, ssum), bo = f2(bout[2 * g], bout[2 * g + 1]);
+          const float2 pg = ssum, bo = f2(bout[2 * g], bout[2 * g + 1]);
           accK = __ffma2_rn(pg, __fadd2_rn(f2(ha0, ha1), bo), accK);
           accB = __ffma2_rn(pg, bo, accB);
           accP = __fadd2_rn(accP, pg);

@@ -272,25 +272,25 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
           const float2 d0 = __fadd2_rn(c0[p], nw0), d1 = __fadd2_rn(c1[p], nw1);
           y[p] = __ffma2_rn(d1, d1, __ffma2_rn(d0, d0, f2(nr[2 * p], nr[2 * p + 1])));
         }
-        const float m = min16(y);
-        const float2 gf = f2s(ex2f(K - hs[k] - m));   // posterior factor of the group
+        // the posterior directly, p = 2^(K - n_sigma - y'), one ex2 per state
+        const float kh = K - hs[k];
         float2 s = f2s(0.f);
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
-          const float2 a = __ffma2_rn(y[p], neg1, f2s(m));
-          const float2 u = f2(ex2f(a.x), ex2f(a.y));
-          s = __fadd2_rn(s, u);
-          const float2 pp = __fmul2_rn(u, gf);
+          const float2 a = __ffma2_rn(y[p], neg1, f2s(kh));
+          const float2 pp = f2(ex2f(a.x), ex2f(a.y));
+          s = __fadd2_rn(s, pp);
           acc0 = __ffma2_rn(pp, c0[p], acc0);
           acc1 = __ffma2_rn(pp, c1[p], acc1);
-          accp = __fadd2_rn(accp, pp);
           if constexpr (ARGMAX) {
             const int q = ((8 * e + k) << 12) | (mid << 4) | (2 * p);
             arg_better(bestp, bestq, pp.x, q);
             arg_better(bestp, bestq, pp.y, q + 1);
           }
         }
-        nout[k] = (m - Rrn) - lg2f(s.x + s.y);
+        accp = __fadd2_rn(accp, s);
+        // negated log rho_{t-1}; +inf (rho = 0) when the group's posterior mass underflows
+        nout[k] = (kh - Rrn) - lg2f(s.x + s.y);
         tmin = fminf(tmin, nout[k]);
       }
       if (t >= 1) {
@@ -540,9 +540,8 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
           const float2 d0 = __fadd2_rn(f2(cw.x, cw.y), nw0), d1 = __fadd2_rn(f2(cw.z, cw.w), nw1);
           y[p] = __ffma2_rn(d1, d1, __ffma2_rn(d0, d0, f2(nr[2 * p], nr[2 * p + 1])));
         }
-        const float m = min16(y);
-        const float gfs = ex2f(K - hsk - m);          // posterior factor of the group
-        const float2 gf = f2s(gfs);
+        // the posterior directly, p = 2^(K - n_sigma - y'), one ex2 per state
+        const float kh = K - hsk;
         const float2 ah = f2s(hak - hbt);             // A - K + gZ
         float2 s = f2s(0.f), num = f2s(0.f);
 #pragma unroll
@@ -557,12 +556,11 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
           const int p = 4 * hf + pl;
           const float4 cw = __ldg(cb + (k * 8 + p) * NT);
           const float2 c0 = f2(cw.x, cw.y), c1 = f2(cw.z, cw.w);
-          const float2 a = __ffma2_rn(y[p], neg1, f2s(m));
-          const float2 u = f2(ex2f(a.x), ex2f(a.y));
-          s = __fadd2_rn(s, u);
+          const float2 a = __ffma2_rn(y[p], neg1, f2s(kh));
+          const float2 pp = f2(ex2f(a.x), ex2f(a.y));
+          s = __fadd2_rn(s, pp);
           const float2 z = __ffma2_rn(g1, c1, __ffma2_rn(g0, c0, f2(bc[2 * p], bc[2 * p + 1])));   // Bc + h
-          num = __ffma2_rn(u, z, num);
-          const float2 pp = __fmul2_rn(u, gf);
+          num = __ffma2_rn(pp, z, num);
           const float2 Gp = __fmul2_rn(pp, __fadd2_rn(z, ah));
           const float2 Gd0 = __fmul2_rn(Gp, __fadd2_rn(c0, nw0));   // G (c0' - w0')
           const float2 Gd1 = __fmul2_rn(Gp, __fadd2_rn(c1, nw1));
@@ -582,10 +580,12 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
         for (int j = 0; j < 2; ++j) gc1[(k * 4 + 2 * hf + j) * NT] = g1v[j];
         }
         const float ss = s.x + s.y;
-        const float nout = (m - Rrn) - lg2f(ss);
-        const float bout = __fdividef(num.x + num.y, ss);
+        // negated log rho_{t-1} and Bc; a group whose posterior mass underflows gets
+        // rho = 0 (+inf) and Bc = 0, moving no posterior by more than that mass
+        const float nout = (kh - Rrn) - lg2f(ss);
+        const float bout = (ss > 0.f) ? __fdividef(num.x + num.y, ss) : 0.f;
         // posterior of the step t-1 group (h, mid): sum over its members of p
-        const float pg = gfs * ss;
+        const float pg = ss;
         accK = fmaf(pg, hak + bout, accK);
         accB = fmaf(pg, bout, accB);
         accP += pg;
