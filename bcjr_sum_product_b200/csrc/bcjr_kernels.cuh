@@ -30,6 +30,7 @@
 // Energies are evaluated in scaled units: with sk = sqrt(log2(e)/T),
 // w' = sk*w and c' = sk*c, log2 psi_t(s) = -||w'_t - c'(s)||^2.
 #pragma once
+#include <cfloat>
 #include <cuda_runtime.h>
 #include <stdint.h>
 

@@ -583,7 +583,7 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
         // negated log rho_{t-1} and Bc; a group whose posterior mass underflows gets
         // rho = 0 (+inf) and Bc = 0, moving no posterior by more than that mass
         const float nout = (kh - Rrn) - lg2f(ss);
-        const float bout = (ss > 0.f) ? __fdividef(num.x + num.y, ss) : 0.f;
+        const float bout = __fdividef(num.x + num.y, fmaxf(ss, FLT_MIN));   // num = 0 when sum p = 0
         // posterior of the step t-1 group (h, mid): sum over its members of p
         const float pg = ss;
         accK = fmaf(pg, hak + bout, accK);
