@@ -601,7 +601,7 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
       const bool last = (t == n - 1);
       const float rA = (t >= 1) ? hist_a[(size_t)(t - 1) * J] : 0.f;   // the forward's reference
       const float hbt = Kt + rA - rB - gzq;
-      float2 accG = f2s(0.f), accGc = f2s(0.f);
+      float2 accGd = f2s(0.f);   // sum_q G (c' - w')
       float2 accK = f2s(0.f), accB = f2s(0.f), accP = f2s(0.f);
       float tmin = INFINITY;
       float4 bvn = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -659,11 +659,10 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
             const float2 z = __ffma2_rn(g2, c2[lo], f2s(bc[lo]));          // Bc + h
             num = __ffma2_rn(pp, z, num);
             const float2 G = __fmul2_rn(pp, __fadd2_rn(z, ah));
-            accG = __fadd2_rn(accG, G);
-            accGc = __ffma2_rn(G, c2[lo], accGc);
+            const float2 Gd = __fmul2_rn(G, __fadd2_rn(c2[lo], nw2));   // G (c' - w')
+            accGd = __fadd2_rn(accGd, Gd);
             float2 gc = f2(gcb[2 * lo], gcb[2 * lo + 1]);
-            gc = __ffma2_rn(gr2, pp, gc);
-            gc = __ffma2_rn(__fmul2_rn(G, __fadd2_rn(c2[lo], nw2)), nc2T, gc);  // + (2/T) G (w - c)
+            gc = __ffma2_rn(Gd, nc2T, __ffma2_rn(gr2, pp, gc));       // + g p + (2/T) G (w - c)
             gcb[2 * lo] = gc.x;
             gcb[2 * lo + 1] = gc.y;
           }
@@ -690,8 +689,7 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
         }
       }
       tmem_wait_st();
-      const float a0 = warp_sum(accGc.x + accGc.y);
-      const float a1 = warp_sum(accG.x + accG.y);
+      const float a0 = warp_sum(accGd.x + accGd.y);
       const float kk = warp_sum(accK.x + accK.y);
       const float kb = warp_sum(accB.x + accB.y);
       const float kp = warp_sum(accP.x + accP.y);
@@ -701,15 +699,14 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
         float* r = rec + (pb * 32 + warp) * 8;
         *reinterpret_cast<float4*>(r) = make_float4(kk, kb, kp, tmin);
         r[4] = a0;
-        r[5] = a1;
       }
       __syncthreads();
       if (tid == 0) {
-        float s0 = 0.f, s1 = 0.f;
+        float s0 = 0.f;
 #pragma unroll
-        for (int w2 = 0; w2 < NT / 32; ++w2) { s0 += rec[(pb * 32 + w2) * 8 + 4]; s1 += rec[(pb * 32 + w2) * 8 + 5]; }
-        // dl/dw_t = (2/T) (sum G c - w_t sum G), c = c'/sk, w_t = -nwt/sk
-        P.grad_w[seq * P.len + t] = P.two_over_T * (s0 + nwt * s1) / P.sk;
+        for (int w2 = 0; w2 < NT / 32; ++w2) s0 += rec[(pb * 32 + w2) * 8 + 4];
+        // dl/dw_t = (2/T) sum_q G (c - w_t) = (2/T) sum_q G (c' - w') / sk
+        P.grad_w[seq * P.len + t] = P.two_over_T * s0 / P.sk;
       }
       Cr -= (double)Rrn;
       {
