@@ -289,7 +289,6 @@ __global__ void __launch_bounds__(kMaxThreads) bcjr_sweep_kernel(SweepParams P) 
         constexpr bool RELOAD = (B * V > 32);
         constexpr int BL = RELOAD ? 1 : B;
         float y[B], z[BL], cc[BL][V];
-        float m = -INFINITY;
 #pragma unroll
         for (int b = 0; b < B; ++b) {
           const int q = (i << D) | b;
@@ -300,7 +299,6 @@ __global__ void __launch_bounds__(kMaxThreads) bcjr_sweep_kernel(SweepParams P) 
 #pragma unroll
           for (int v = 0; v < V; ++v) { float d = wt[v] - c[v]; acc = fmaf(-d, d, acc); }
           y[b] = acc;
-          m = fmaxf(m, acc);
           if constexpr (!RELOAD) {
 #pragma unroll
             for (int v = 0; v < V; ++v) cc[b][v] = c[v];
@@ -312,13 +310,13 @@ __global__ void __launch_bounds__(kMaxThreads) bcjr_sweep_kernel(SweepParams P) 
             }
           }
         }
-        const float gf = ex2f(m + lsig + K);  // posterior factor of the group
+        // the posterior directly, p = 2^(log2 sigma + y + K), one ex2 per state
+        const float kh = lsig + K;
         float sum = 0.f, num = 0.f;
 #pragma unroll
         for (int b = 0; b < B; ++b) {
-          const float u = ex2f(y[b] - m);
-          sum += u;
-          const float p = u * gf;
+          const float p = ex2f(y[b] + kh);
+          sum += p;
           const int q = (i << D) | b;
           float c[V], zb = 0.f;
           if constexpr (RELOAD) {
@@ -340,7 +338,7 @@ __global__ void __launch_bounds__(kMaxThreads) bcjr_sweep_kernel(SweepParams P) 
             np_[V] += p;
             arg_better(bestp, bestq, p, q);
           } else {
-            num = fmaf(u, zb, num);
+            num = fmaf(p, zb, num);
             const float G = p * (asig + zb - hb);
             np_[V] += G;
             float* gq = gc_seq + (size_t)q * V;
@@ -354,13 +352,15 @@ __global__ void __launch_bounds__(kMaxThreads) bcjr_sweep_kernel(SweepParams P) 
           }
         }
         if (t >= 1) {
-          const float l = m + lg2f(sum) - Rr;
+          // log2 rho_{t-1}(i) = lg2 sum p - (log2 sigma + K); a group whose posterior mass
+          // underflows gets rho = 0 (-inf) and Bc = 0, moving no posterior by more than that mass
+          const float l = lg2f(sum) - kh - Rr;
           rnext[i] = l;
           tmax = fmaxf(tmax, l);
           if constexpr (VJP) {
-            const float bn = __fdividef(num, sum);
+            const float bn = (sum > 0.f) ? __fdividef(num, sum) : 0.f;
             bnext[i] = bn;
-            const float pg = gf * sum;   // posterior of group i at step t-1
+            const float pg = sum;   // posterior of group i at step t-1
             np_[NP] = fmaf(pg, asig + bn, np_[NP]);
             np_[NP + 1] = fmaf(pg, bn, np_[NP + 1]);
             np_[NP + 2] += pg;
