@@ -123,8 +123,12 @@ struct Arena {
   }
 };
 
-int threads_for(int J) {
-  int t = J < 32 ? 32 : (J > bcjr::kMaxThreads ? bcjr::kMaxThreads : J);
+// Generic kernels: about 32 states per thread per step (J groups of B members),
+// 32 to 512 threads.  Small trellises then run several small CTAs per SM instead
+// of one large CTA whose per-step barrier and reductions outweigh its work.
+int threads_for(int J, int B) {
+  const long w = (long)J * B / 32;
+  const int t = w < 32 ? 32 : (w > bcjr::kMaxThreads ? bcjr::kMaxThreads : (int)w);
   return (t + 31) / 32 * 32;
 }
 
@@ -294,7 +298,7 @@ int run_sweep(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   if (use_l16v2(sh)) return run_l16v2<MODE>(sh, a, st);
   SweepKernel kern = pick_sweep<MODE>(sh.V, sh.D);
   if (!kern) return BCJR_ERR_UNSUPPORTED;
-  const int threads = threads_for(sh.J);
+  const int threads = threads_for(sh.J, sh.B);
   const int NPT = sh.V + 1 + (VJP ? 3 : 0);   // per-warp partials per step
   size_t fixed = sizeof(float) * ((size_t)sh.n * sh.V * (VJP ? 2 : 1) + 64 + 64 * NPT + 64 + 64);
   size_t state_bytes = sizeof(float) * (size_t)sh.J * (VJP ? 4 : 2);
@@ -397,7 +401,7 @@ int run_viterbi(const Shape& sh, const float* w, const float* c, int32_t* out_st
   if (sh.L == 16 && sh.D == 2 && sh.V == 1 && !generic_only()) return run_viterbi_l16(sh, w, c, out_states, out_cost, st);
   ViterbiKernel kern = pick_viterbi(sh.V, sh.D);
   if (!kern) return BCJR_ERR_UNSUPPORTED;
-  const int threads = threads_for(sh.J);
+  const int threads = threads_for(sh.J, sh.B);
   size_t fixed = sizeof(float) * ((size_t)sh.n * sh.V + 64);
   size_t state_bytes = sizeof(float) * (size_t)sh.J * 2;
   const bool in_smem = fixed + state_bytes <= kMaxDynSmem;
@@ -612,7 +616,7 @@ extern "C" int bcjr_soft_codeword_noalloc(const float* w, int64_t n_seq, int64_t
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   SweepKernel kern = pick_sweep<bcjr::MODE_SOFT>(sh.V, sh.D);
   if (!kern) return BCJR_ERR_UNSUPPORTED;
-  const int threads = threads_for(sh.J);
+  const int threads = threads_for(sh.J, sh.B);
   const int NP = sh.V + 1;
   const size_t fixed = sizeof(float) * ((size_t)sh.n * sh.V + 64 + 64 * NP + 64 + 64);
   const size_t state_bytes = sizeof(float) * (size_t)sh.J * 2;
