@@ -61,7 +61,7 @@ LEDGER = LEDGERS[(2, 1)]
 # profiles/soft_kernel_qtip16.md); set to None whenever the kernel changes.
 # (A 16-sequence capture of the V=2 kernels keeps their histories in L2, so it
 # does not scale to a full launch; their traffic is reported as null.)
-TRAFFIC_PER_SEQ = {"vjp": 1003.29e6 / 16, "soft": 448.17e6 / 16}
+TRAFFIC_PER_SEQ = {"vjp": 1000.14e6 / 16, "soft": 443.19e6 / 16}
 FP32_PER_CLK_SM = 128.0   # FFMA lanes per SM per clock (measured 123.5 FFMA, 126 FFMA2 on this machine)
 MUFU_PER_CLK_SM = 16.0    # ex2 per SM per clock (measured 15.99 on this machine)
 N_SM = 148
