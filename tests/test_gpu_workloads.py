@@ -130,3 +130,9 @@ def test_layer_workload():
     rows = _rows(wl.n_seq, 8, 8)
     _check_rows(inp, T, res, rows)
     _translation_identity(inp, res)
+    # the hard limit over the whole workload, bit-exact on the sampled rows
+    states, cost = lib.viterbi_decode(inp.w.to(DEV), inp.c.to(DEV), wl.L, wl.k, wl.V)
+    torch.cuda.synchronize()
+    ref = oracle.viterbi(inp.w[rows], inp.c, wl.L, wl.k, wl.V)
+    np.testing.assert_array_equal(states.cpu().numpy()[rows], ref["states"])
+    np.testing.assert_array_equal(cost.cpu().numpy()[rows], ref["cost"])
