@@ -13,7 +13,7 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-@pytest.mark.parametrize("L,k,V,T", [(8, 2, 1, 0.3), (10, 2, 2, 0.1), (16, 2, 1, 0.05)])
+@pytest.mark.parametrize("L,k,V,T", [(8, 2, 1, 0.3), (10, 2, 2, 0.1), (16, 2, 1, 0.05), (16, 2, 2, 0.05)])
 def test_qat_step_matches_oracle(L, k, V, T):
     n_seq = 12 if L < 16 else 3
     target, c, _ = I.random_case(L, k, V, n_seq, 32 * V, seed=400 + L + V)
