@@ -57,8 +57,8 @@ LEDGERS = {
 }
 LEDGER = LEDGERS[(2, 1)]
 # DRAM bytes per sequence (read + write) of each L=16, V=1 sweep kernel, from one
-# ncu capture of 16 qtip sequences (profiles/vjp_kernel_qtip16.md,
-# profiles/soft_kernel_qtip16.md); set to None whenever the kernel changes.
+# ncu capture of 16 qtip sequences (one sequence per CTA, the same per-SM
+# history traffic as a full launch); set to None whenever the kernel changes.
 # (A 16-sequence capture of the V=2 kernels keeps their histories in L2, so it
 # does not scale to a full launch; their traffic is reported as null.)
 TRAFFIC_PER_SEQ = {"vjp": 1000.14e6 / 16, "soft": 443.19e6 / 16}
