@@ -175,7 +175,7 @@ def run_reference(args):
     T = args.temp if args.temp is not None else wl.temps[0]
     do_vjp = "vjp" in wl.calls
     cores = os.cpu_count() or 1
-    n_rows = max(1, min(cores, 16, wl.n_seq))
+    n_rows = max(1, min(cores, 128, wl.n_seq))   # one sequence per host core
     inp = I.make(args.workload, rows=list(range(n_rows)))
     import oracle
 
@@ -420,7 +420,7 @@ def main():
         line_note = None
     if world == 1 and not args.no_cpu_baseline:
         cores = os.cpu_count() or 1
-        cpu = cpu_baseline(wl, inp, max(1, min(cores, 16, n_seq)), T, do_vjp)
+        cpu = cpu_baseline(wl, inp, max(1, min(cores, 128, n_seq)), T, do_vjp)   # one sequence per host core
 
     metric = metric_for(wl, do_vjp)
     if args.qat:
