@@ -129,20 +129,33 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def cpu_baseline(wl, inp, n_rows: int, T: float, do_vjp: bool):
-    """The oracle as it stands, on n_rows sequences of the workload, all host cores."""
-    import oracle
+def oracle_sample_rows(wl, n_avail: int) -> int:
+    """Sequences (= oracle threads) for a timed CPU sample: one per host core, at
+    most 128, and within a memory budget (each oracle thread holds about three
+    n x 2^L fp64 arrays): 1/16 of physical memory, at most 32 GB."""
     cores = os.cpu_count() or 1
+    per_thread = 3 * wl.n_steps * wl.S * 8
+    try:
+        phys = os.sysconf("SC_PAGE_SIZE") * os.sysconf("SC_PHYS_PAGES")
+    except (ValueError, OSError, AttributeError):
+        phys = 64 << 30
+    budget = min(phys // 16, 32 << 30)
+    return max(1, min(cores, 128, n_avail, budget // per_thread))
+
+
+def cpu_baseline(wl, inp, n_rows: int, T: float, do_vjp: bool):
+    """The oracle as it stands, on n_rows sequences of the workload, one host thread each."""
+    import oracle
     rows = list(range(n_rows))
     w = inp.w[rows].contiguous()
     t0 = time.perf_counter()
-    oracle.soft(w, inp.c, wl.L, wl.k, wl.V, T, nthreads=cores)
+    oracle.soft(w, inp.c, wl.L, wl.k, wl.V, T, nthreads=n_rows)
     if do_vjp:
-        oracle.vjp(w, inp.c, wl.L, wl.k, wl.V, T, inp.g[rows].contiguous(), nthreads=cores)
+        oracle.vjp(w, inp.c, wl.L, wl.k, wl.V, T, inp.g[rows].contiguous(), nthreads=n_rows)
     dt = time.perf_counter() - t0
     units = n_rows * wl.n_steps * wl.S
     what = "soft codeword + VJP" if do_vjp else "soft codeword"
-    return {"value": units / dt, "unit": UNIT, "cores": min(cores, n_rows), "kind": "oracle",
+    return {"value": units / dt, "unit": UNIT, "cores": n_rows, "kind": "oracle",
             "sample": f"{n_rows} of {wl.n_seq} sequences of the {wl.name} workload, {what}, "
                       f"fp64 C oracle with OpenMP over sequences; {dt:.1f} s"}
 
@@ -174,15 +187,14 @@ def run_reference(args):
     wl = I.WORKLOADS[args.workload]
     T = args.temp if args.temp is not None else wl.temps[0]
     do_vjp = "vjp" in wl.calls
-    cores = os.cpu_count() or 1
-    n_rows = max(1, min(cores, 128, wl.n_seq))   # one sequence per host core
+    n_rows = oracle_sample_rows(wl, wl.n_seq)   # one sequence per oracle thread
     inp = I.make(args.workload, rows=list(range(n_rows)))
     import oracle
 
     def step():
-        oracle.soft(inp.w, inp.c, wl.L, wl.k, wl.V, T, nthreads=cores)
+        oracle.soft(inp.w, inp.c, wl.L, wl.k, wl.V, T, nthreads=n_rows)
         if do_vjp:
-            oracle.vjp(inp.w, inp.c, wl.L, wl.k, wl.V, T, inp.g, nthreads=cores)
+            oracle.vjp(inp.w, inp.c, wl.L, wl.k, wl.V, T, inp.g, nthreads=n_rows)
 
     for _ in range(args.warmup):
         step()
@@ -199,7 +211,7 @@ def run_reference(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": describe(wl, T, do_vjp), "sample_sequences": n_rows},
             "weights_per_s": n_rows * wl.seq_len / dt,
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(cores, n_rows), "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": n_rows, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -419,8 +431,7 @@ def main():
     else:
         line_note = None
     if world == 1 and not args.no_cpu_baseline:
-        cores = os.cpu_count() or 1
-        cpu = cpu_baseline(wl, inp, max(1, min(cores, 128, n_seq)), T, do_vjp)   # one sequence per host core
+        cpu = cpu_baseline(wl, inp, oracle_sample_rows(wl, n_seq), T, do_vjp)
 
     metric = metric_for(wl, do_vjp)
     if args.qat:
