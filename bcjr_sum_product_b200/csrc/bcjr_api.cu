@@ -12,6 +12,7 @@
 #include "bcjr.h"
 #include "bcjr_kernels.cuh"
 #include "bcjr_l16.cuh"
+#include "bcjr_l16c.cuh"
 #include "bcjr_l16v2.cuh"
 
 namespace {
@@ -191,13 +192,104 @@ struct SweepArgs {
   float* grad_c;
 };
 
+// Measured alternatives of the L = 16, k = 2, V = 1 kernels, selected per call.
+// BCJR_L16_VJP=cluster runs the VJP on clusters of two CTAs (bcjr_l16c.cuh)
+// instead of one CTA per sequence.  The backward sweeps run in posterior space
+// for the soft codeword and in log domain for the VJP (the faster of the two for
+// each); BCJR_L16_BWD=post or =log selects one of them for both.
+bool l16_vjp_cluster() {
+  const char* e = std::getenv("BCJR_L16_VJP");
+  return e && std::strcmp(e, "cluster") == 0;
+}
+bool l16_posterior_backward(bool vjp) {
+  const char* e = std::getenv("BCJR_L16_BWD");
+  if (e && std::strcmp(e, "post") == 0) return true;
+  if (e && std::strcmp(e, "log") == 0) return false;
+  return !vjp;
+}
+
+// L = 16, D = 2, V = 1 VJP on clusters of two CTAs (bcjr_l16c.cuh).  Returns
+// BCJR_ERR_UNSUPPORTED, with nothing launched, when no cluster fits an SM pair.
+int run_l16c_vjp(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
+  namespace K = bcjr::l16c;
+  const size_t smem = sizeof(float) * K::smem_floats(sh.n);
+  if (smem > kMaxDynSmem) return BCJR_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(K::vjp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
+    cudaGetLastError();
+    return BCJR_ERR_UNSUPPORTED;
+  }
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = K::NC;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(K::NT, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int dev = 0, nsm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return BCJR_ERR_CUDA;
+  }
+  cfg.gridDim = dim3((unsigned)(K::NC * (nsm / K::NC)), 1, 1);
+  int max_clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&max_clusters, K::vjp_kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return BCJR_ERR_UNSUPPORTED;
+  }
+  if (max_clusters < 1) return BCJR_ERR_UNSUPPORTED;
+  int ncl = (int)std::min<int64_t>(max_clusters, sh.n_seq);
+  cap_grid_by_memory(&ncl, sizeof(float) * (size_t)K::NC * 2 * sh.n * K::JL +
+                               (sizeof(double) + sizeof(float)) * sh.n + sizeof(double) * K::S);
+  K::Params P{};
+  auto layout = [&](Arena& ar) {
+    P.cs_tm = ar.take<float>(K::S);
+    P.hist_l = ar.take<float>((size_t)K::NC * ncl * sh.n * K::JL);
+    P.hist_a = ar.take<float>((size_t)K::NC * ncl * sh.n * K::JL);
+    P.hist_c = ar.take<double>((size_t)ncl * sh.n);
+    P.hist_r = ar.take<float>((size_t)ncl * sh.n);
+    P.gc_part = ar.take<double>((size_t)ncl * K::S);
+  };
+  Arena sizing;
+  layout(sizing);
+  void* mem = nullptr;
+  if (int arc = scratch_alloc(&mem, sizing.off, st)) return arc;
+  Arena ar;
+  ar.base = static_cast<char*>(mem);
+  layout(ar);
+  P.w = a.w; P.gsoft = a.gsoft; P.gZ = a.gZ; P.grad_w = a.grad_w;
+  P.n_seq = sh.n_seq; P.len = sh.len; P.n = sh.n;
+  P.sk = (float)std::sqrt(1.4426950408889634 / (double)a.T);
+  P.two_over_T = (float)(2.0 / (double)a.T);
+  cfg.gridDim = dim3((unsigned)(K::NC * ncl), 1, 1);
+  bcjr::l16::make_block_codebook<<<K::S / 256, 256, 0, st>>>(a.c, P.sk, const_cast<float*>(P.cs_tm));
+  cudaError_t ke = cudaLaunchKernelEx(&cfg, K::vjp_kernel, P);
+  if (ke == cudaSuccess) bcjr::l16::reduce_block_gc<<<K::S / 256, 256, 0, st>>>(P.gc_part, ncl, a.grad_c);
+  cudaError_t le = cudaGetLastError();
+  cudaError_t fe = cudaFreeAsync(mem, st);
+  if (ke != cudaSuccess || le != cudaSuccess || fe != cudaSuccess) return BCJR_ERR_CUDA;
+  return BCJR_OK;
+}
+
 // L = 16, D = 2, V = 1: the block-layout kernel of bcjr_l16.cuh.
 template <int MODE>
 int run_l16(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   namespace K = bcjr::l16;
   constexpr bool VJP = MODE == bcjr::MODE_VJP;
-  void (*kern)(K::Params) = K::vjp_kernel;
-  if (!VJP) kern = a.out_argmax ? K::soft_kernel<true> : K::soft_kernel<false>;
+  if (VJP && l16_vjp_cluster()) {
+    const int rc = run_l16c_vjp(sh, a, st);
+    if (rc != BCJR_ERR_UNSUPPORTED) return rc;
+  }
+  const bool post = l16_posterior_backward(VJP);
+  void (*kern)(K::Params) = post ? K::vjp_kernel<true> : K::vjp_kernel<false>;
+  if (!VJP) {
+    if (post) kern = a.out_argmax ? K::soft_kernel<true, true> : K::soft_kernel<false, true>;
+    else kern = a.out_argmax ? K::soft_kernel<true, false> : K::soft_kernel<false, false>;
+  }
   // state ping-pong, per-warp partials, TMEM slot, per-step weights (and gradients)
   const size_t smem = sizeof(float) * ((size_t)2 * K::J + (VJP ? 2 * 32 * 8 : 64 + 2 * 32 * 2 + 64 + 64) + 4 +
                                        (VJP ? 2 : 1) * (size_t)sh.n);
@@ -205,7 +297,7 @@ int run_l16(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   int grid = 0;
   int rc = grid_for(kern, K::NT, smem, sh.n_seq, &grid);
   if (rc != BCJR_OK) return rc;
-  cap_grid_by_memory(&grid, sizeof(float) * (size_t)sh.n * K::J * (VJP ? 2 : 1) + sizeof(double) * sh.n +
+  cap_grid_by_memory(&grid, sizeof(float) * (size_t)sh.n * K::J * (VJP ? 2 : 1) + (sizeof(double) + sizeof(float)) * sh.n +
                                 (VJP ? sizeof(float) * 2 * K::J + sizeof(double) * K::S : 0));
   K::Params P{};
   auto layout = [&](Arena& ar) {
@@ -213,6 +305,7 @@ int run_l16(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
     P.hist_l = ar.take<float>((size_t)grid * sh.n * K::J);
     P.hist_a = VJP ? ar.take<float>((size_t)grid * sh.n * K::J) : nullptr;
     P.hist_c = ar.take<double>((size_t)grid * sh.n);
+    P.hist_rn = ar.take<float>((size_t)grid * sh.n);
     P.bc_g = VJP ? ar.take<float>((size_t)grid * 2 * K::J) : nullptr;
     P.gc_part = VJP ? ar.take<double>((size_t)grid * K::S) : nullptr;
   };

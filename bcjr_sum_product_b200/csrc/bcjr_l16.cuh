@@ -30,6 +30,15 @@
 #pragma once
 #include "bcjr_kernels.cuh"
 
+// Prefetch distances of the VJP backward: codewords two units (8 states)
+// ahead, history vectors one block ahead.
+#ifndef BCJR_VJP_CB_AHEAD
+#define BCJR_VJP_CB_AHEAD 2
+#endif
+#ifndef BCJR_VJP_HOUT_AHEAD
+#define BCJR_VJP_HOUT_AHEAD 1
+#endif
+
 namespace bcjr {
 namespace l16 {
 
@@ -50,7 +59,8 @@ struct Params {
   double* gc_part;       // [grid][65536] block-major (VJP)
   float* hist_l;         // [grid][n][J]
   float* hist_a;         // [grid][n][J] (VJP)
-  double* hist_c;        // [grid][n]
+  double* hist_c;        // [grid][n]  fp64 offsets of the forward steps
+  float* hist_rn;        // [grid][n]  re-centring value of each forward step
   float* bc_g;           // [grid][2][J] (VJP backward ping-pong)
   int64_t n_seq, len;
   int n;
@@ -176,6 +186,23 @@ __global__ void reduce_block_gc(const double* __restrict__ part, int nparts, flo
 // every line an FFMA/FADD without negations.  Pairs (h, h+1) share one f32x2
 // lane pair: in the forward they are two members of one group, in the
 // backward two groups with the same member.
+//
+// The forward stores every step's group values n_t(j) in group order [t][j];
+// the backward of block mid at step t reads its own four outputs n_t((mid << 2) | lo)
+// (one 16-byte vector) and its four inputs n_{t-1}((h << 12) | mid) (four
+// scalars that consecutive threads read from consecutive addresses).
+//
+// Two backward sweeps (template parameter POST):
+//  * posterior space (POST): with u_t(q) = alpha_t(q) / sigma_t(q mod J), the
+//    forward weight of q within its group, and P_t(j) the posterior mass of
+//    forward group j at step t,
+//        p_t(q) = u_t(q) P_t(q mod J),   P_{t-1}(i) = sum_lo p_t((i << 2) | lo),
+//        log2 u_t(q) = n_t(q mod J) + Rn_t - (d_t(q)^2 + n_{t-1}(q >> 2)),
+//    where Rn_t is the re-centring value of forward step t: one ex2 and one
+//    multiply per state, linear sums per group, no logarithm; the exchanged
+//    values are probabilities (no range problem at any temperature);
+//  * log domain: p = 2^(K - n_sigma - y') with the negated log rho exchanged,
+//    one ex2 per state plus one lg2 per group.
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
 __device__ __forceinline__ float2 f2s(float a) { return make_float2(a, a); }
 
@@ -194,7 +221,31 @@ __device__ __forceinline__ float bfly16_sum(float v) {
   return v;
 }
 
-template <bool ARGMAX>
+// One forward group of the soft pass: x_h = d_h^2 + n_h for the four members
+// (h = 0..3 in two lane pairs); returns the negated log2 of sum_h 2^(-x_h)
+// re-centred by Rn.  The smallest x contributes 2^0 = 1 exactly, so only the
+// three others need an ex2: a min/max network picks them.
+__device__ __forceinline__ float soft_group(float2 x01, float2 x23, float Rn) {
+  const float l01 = fminf(x01.x, x01.y), h01 = fmaxf(x01.x, x01.y);
+  const float l23 = fminf(x23.x, x23.y), h23 = fmaxf(x23.x, x23.y);
+  const float m = fminf(l01, l23), M = fmaxf(l01, l23);
+  const float2 a = __ffma2_rn(f2(h01, h23), f2s(-1.f), f2s(m));
+  const float s = (1.f + ex2f(m - M)) + (ex2f(a.x) + ex2f(a.y));
+  return (m - Rn) - lg2f(s);
+}
+
+// n_{tt-1}((h << 12) | mid) for h = 0..3 (zero for tt = 0: free start)
+__device__ __forceinline__ float4 hist_in(const float* hist, int tt, int mid) {
+  if (tt < 1) return make_float4(0.f, 0.f, 0.f, 0.f);
+  const float* p = hist + (size_t)(tt - 1) * J + mid;
+  return make_float4(p[0], p[1 << HB], p[2 << HB], p[3 << HB]);
+}
+// n_tt((mid << 2) | lo) for lo = 0..3
+__device__ __forceinline__ float4 hist_out(const float* hist, int tt, int mid) {
+  return reinterpret_cast<const float4*>(hist + (size_t)tt * J)[mid];
+}
+
+template <bool ARGMAX, bool POST>
 __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
   constexpr int NP = 2;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -202,7 +253,7 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
   const int n = P.n;
 
   extern __shared__ __align__(16) float smem[];
-  float* sb = smem;                                    // [2][J] negated state ping-pong
+  float* sb = smem;                                    // [2][J] forward values / backward messages
   float* lb[2] = {sb, sb + J};
   float* wmin = sb + 2 * J;                            // [2][32]
   float* part = wmin + 64;                             // [2][32][NP]
@@ -211,8 +262,9 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
   uint32_t* tslot = reinterpret_cast<uint32_t*>(aidx + 64);  // [4]
   float* wsc = reinterpret_cast<float*>(tslot + 4);    // n
 
-  float* hist = P.hist_l + (size_t)blockIdx.x * n * J;   // negated forward values
+  float* hist = P.hist_l + (size_t)blockIdx.x * n * J;   // [n][J] negated forward values, group order
   double* hist_c = P.hist_c + (size_t)blockIdx.x * n;
+  float* hist_rn = P.hist_rn + (size_t)blockIdx.x * n;
   const float2 neg1 = f2s(-1.f);
 
   if (warp == 0) tmem_alloc512(tslot);
@@ -253,35 +305,30 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
         } else {
           np01 = f2(nprev[(0 << HB) | mid], nprev[(1 << HB) | mid]);
           np23 = f2(nprev[(2 << HB) | mid], nprev[(3 << HB) | mid]);
-          // history of step t-1 in block-major order [mid][h]: what the backward reads per block
-          reinterpret_cast<float4*>(hist + (size_t)(t - 1) * J)[mid] = make_float4(np01.x, np01.y, np23.x, np23.y);
         }
         float out[4];
 #pragma unroll
         for (int lo = 0; lo < 4; ++lo) {
           const float2 d01 = __fadd2_rn(f2(cb[bidx(0, lo)], cb[bidx(1, lo)]), nw2);
           const float2 d23 = __fadd2_rn(f2(cb[bidx(2, lo)], cb[bidx(3, lo)]), nw2);
-          const float2 x01 = __ffma2_rn(d01, d01, np01);
-          const float2 x23 = __ffma2_rn(d23, d23, np23);
-          const float m = fminf(fminf(x01.x, x01.y), fminf(x23.x, x23.y));
-          const float2 a01 = __ffma2_rn(x01, neg1, f2s(m));
-          const float2 a23 = __ffma2_rn(x23, neg1, f2s(m));
-          const float2 s2 = __fadd2_rn(f2(ex2f(a01.x), ex2f(a01.y)), f2(ex2f(a23.x), ex2f(a23.y)));
-          out[lo] = (m - Rn) - lg2f(s2.x + s2.y);
+          out[lo] = soft_group(__ffma2_rn(d01, d01, np01), __ffma2_rn(d23, d23, np23), Rn);
         }
         tmin = fminf(tmin, fminf(fminf(out[0], out[1]), fminf(out[2], out[3])));
-        reinterpret_cast<float4*>(ncur)[mid] = make_float4(out[0], out[1], out[2], out[3]);
+        const float4 ov = make_float4(out[0], out[1], out[2], out[3]);
+        reinterpret_cast<float4*>(ncur)[mid] = ov;
+        reinterpret_cast<float4*>(hist + (size_t)t * J)[mid] = ov;
       }
       tmin = -warp_max(-tmin);
       if (lane == 0) wmin[(t & 1) * 32 + warp] = tmin;
-      if (tid == 0) hist_c[t] = C;
+      if (tid == 0) { hist_c[t] = C; hist_rn[t] = Rn; }
       __syncthreads();
       Rn = bfly16_min(wmin[(t & 1) * 32 + (lane & 15)]);
     }
-    // log2 Z = -Rn + log2 sum_j 2^(Rn - stored_j) + C
+    // log2 Z = -Rn + log2 sum_j 2^(Rn - stored_j) + C; the posterior space
+    // backward starts from P_{n-1}(j) = 2^(Rn - stored_j) / sum, written in place
     double l2Z;
     {
-      const float* nfin = lb[(n - 1) & 1];
+      float* nfin = lb[(n - 1) & 1];
       float s0 = 0.f;
       for (int j = tid; j < J; j += NT) s0 += ex2f(Rn - nfin[j]);
       s0 = warp_sum(s0);
@@ -292,110 +339,187 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
       for (int w2 = 0; w2 < nwarps; ++w2) a0 += part[w2 * NP];
       l2Z = -(double)Rn + log2((double)a0) + C;
       if (tid == 0 && P.out_logZ) P.out_logZ[seq] = (float)(l2Z * 0.69314718055994530942);
+      if constexpr (POST) {
+        const float inv = 1.f / a0;
+        for (int j = tid; j < J; j += NT) nfin[j] = ex2f(Rn - nfin[j]) * inv;
+      }
       __syncthreads();
     }
 
     // ------------------------------------------------------------ backward
-    float Rrn = 0.f;
-    double Cr = 0.0;   // log2 beta_t = -stored + Cr_t
-    // block kk of step tt reads step tt-1's values (free start: 0 for tt = 0)
-    auto hist_at = [&](int tt, int kk) -> float4 {
-      return (tt >= 1) ? reinterpret_cast<const float4*>(hist + (size_t)(tt - 1) * J)[tid + NT * kk]
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
-    };
-    float4 hsn = hist_at(n - 1, 0), hsm = hist_at(n - 1, 1);
-    for (int t = n - 1; t >= 0; --t) {
-      if (warp == 0) prefetch_history(hist, t, lane);
-      const float* ncur = lb[t & 1];
-      float* nnext = lb[(t + 1) & 1];
-      const float2 nw2 = f2s(wsc[t]);
-      const double Csig = (t >= 1) ? hist_c[t - 1] : 0.0;
-      const float K = (float)(Csig + Cr - l2Z);
-      const bool last = (t == n - 1);
-      float2 accc = f2s(0.f), accp = f2s(0.f);
-      float bestp = -1.f;
-      int bestq = 0x7fffffff;
-      float tmin = INFINITY;
+    if constexpr (POST) {
+      // block kk of step tt: its inputs (scalars) and outputs (vector), one block ahead
+      float4 hin_n = hist_in(hist, n - 1, tid), hout_n = hist_out(hist, n - 1, tid);
+      for (int t = n - 1; t >= 0; --t) {
+        if (warp == 0) prefetch_history(hist, t, lane);
+        const float* pcur = lb[t & 1];
+        float* pnext = lb[(t + 1) & 1];
+        const float2 nw2 = f2s(wsc[t]);
+        const float rn = hist_rn[t];
+        float2 accc = f2s(0.f), accp = f2s(0.f);
+        float bestp = -1.f;
+        int bestq = 0x7fffffff;
 #pragma unroll
-      for (int k = 0; k < KB; ++k) {
-        const int mid = tid + NT * k;
-        float cb[16];
-        tmem_ld16(tbase + 16 * k, cb);
-        const float hs[4] = {hsn.x, hsn.y, hsn.z, hsn.w};
-        {
-          const int nt = (k + 2 < KB) ? t : t - 1, nk = (k + 2 < KB) ? k + 2 : k + 2 - KB;
-          hsn = hsm;
-          hsm = hist_at(nt, nk);
-        }
-        float nr[4];
-        if (last) {
-          nr[0] = nr[1] = nr[2] = nr[3] = 0.f;
-        } else {
-          const float4 rv = reinterpret_cast<const float4*>(ncur)[mid];
-          nr[0] = rv.x; nr[1] = rv.y; nr[2] = rv.z; nr[3] = rv.w;
-        }
-        float nout[4];
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {          // groups h = 2g, 2g+1 side by side
-          float2 y[4];
-#pragma unroll
-          for (int lo = 0; lo < 4; ++lo) {
-            const float2 d = __fadd2_rn(f2(cb[bidx(2 * g, lo)], cb[bidx(2 * g + 1, lo)]), nw2);
-            y[lo] = __ffma2_rn(d, d, f2s(nr[lo]));
+        for (int k = 0; k < KB; ++k) {
+          const int mid = tid + NT * k;
+          float cb[16];
+          tmem_ld16(tbase + 16 * k, cb);
+          const float4 hi4 = hin_n, ho4 = hout_n;
+          if (k + 1 < KB) {
+            hin_n = hist_in(hist, t, mid + NT);
+            hout_n = hist_out(hist, t, mid + NT);
+          } else if (t >= 1) {
+            hin_n = hist_in(hist, t - 1, tid);
+            hout_n = hist_out(hist, t - 1, tid);
           }
-          // the posterior directly, p = 2^(K - n_sigma - y'), one ex2 per state
-          const float2 kh = __fadd2_rn(f2s(K), f2(-hs[2 * g], -hs[2 * g + 1]));
-          float2 ssum = f2s(0.f);
+          const float4 pv = reinterpret_cast<const float4*>(pcur)[mid];
+          const float pl[4] = {pv.x, pv.y, pv.z, pv.w};
+          const float nr[4] = {ho4.x + rn, ho4.y + rn, ho4.z + rn, ho4.w + rn};
+          float pn[4];
 #pragma unroll
-          for (int lo = 0; lo < 4; ++lo) {
-            const float2 a = __ffma2_rn(y[lo], neg1, kh);
-            const float2 pp = f2(ex2f(a.x), ex2f(a.y));
-            ssum = __fadd2_rn(ssum, pp);
-            accc = __ffma2_rn(pp, f2(cb[bidx(2 * g, lo)], cb[bidx(2 * g + 1, lo)]), accc);
-            if constexpr (ARGMAX) {
-              arg_better(bestp, bestq, pp.x, ((2 * g) << 14) | (mid << 2) | lo);
-              arg_better(bestp, bestq, pp.y, ((2 * g + 1) << 14) | (mid << 2) | lo);
+          for (int g = 0; g < 2; ++g) {          // groups h = 2g, 2g+1 side by side
+            const float2 np2 = g ? f2(hi4.z, hi4.w) : f2(hi4.x, hi4.y);
+            float2 ssum = f2s(0.f);
+#pragma unroll
+            for (int lo = 0; lo < 4; ++lo) {
+              const float2 c2 = f2(cb[bidx(2 * g, lo)], cb[bidx(2 * g + 1, lo)]);
+              const float2 d = __fadd2_rn(c2, nw2);
+              const float2 a = __ffma2_rn(__ffma2_rn(d, d, np2), neg1, f2s(nr[lo]));
+              const float2 pp = __fmul2_rn(f2(ex2f(a.x), ex2f(a.y)), f2s(pl[lo]));
+              ssum = __fadd2_rn(ssum, pp);
+              accc = __ffma2_rn(pp, c2, accc);
+              if constexpr (ARGMAX) {
+                arg_better(bestp, bestq, pp.x, ((2 * g) << 14) | (mid << 2) | lo);
+                arg_better(bestp, bestq, pp.y, ((2 * g + 1) << 14) | (mid << 2) | lo);
+              }
             }
+            accp = __fadd2_rn(accp, ssum);
+            pn[2 * g] = ssum.x;
+            pn[2 * g + 1] = ssum.y;
           }
-          accp = __fadd2_rn(accp, ssum);
-          // negated log rho_{t-1} = (K - n_sigma) - lg2 sum p (+inf, i.e. rho = 0, when the
-          // group's posterior mass underflows; it then moves no posterior by more than that mass)
-          nout[2 * g] = (kh.x - Rrn) - lg2f(ssum.x);
-          nout[2 * g + 1] = (kh.y - Rrn) - lg2f(ssum.y);
+          if (t >= 1) {
+#pragma unroll
+            for (int h = 0; h < 4; ++h) pnext[(h << HB) | mid] = pn[h];
+          }
         }
-        if (t >= 1) {
-#pragma unroll
-          for (int h = 0; h < 4; ++h) nnext[(h << HB) | mid] = nout[h];
-          tmin = fminf(tmin, fminf(fminf(nout[0], nout[1]), fminf(nout[2], nout[3])));
+        float a0 = warp_sum(accc.x + accc.y);
+        float a1 = warp_sum(accp.x + accp.y);
+        if constexpr (ARGMAX) warp_argmax(bestp, bestq);
+        const int pb = t & 1;
+        if (lane == 0) {
+          part[(pb * 32 + warp) * NP] = a0;
+          part[(pb * 32 + warp) * NP + 1] = a1;
+          if constexpr (ARGMAX) { apart[pb * 32 + warp] = bestp; aidx[pb * 32 + warp] = bestq; }
         }
-      }
-      float a0 = warp_sum(accc.x + accc.y);
-      float a1 = warp_sum(accp.x + accp.y);
-      tmin = -warp_max(-tmin);
-      if constexpr (ARGMAX) warp_argmax(bestp, bestq);
-      const int pb = t & 1;
-      if (lane == 0) {
-        part[(pb * 32 + warp) * NP] = a0;
-        part[(pb * 32 + warp) * NP + 1] = a1;
-        wmin[pb * 32 + warp] = tmin;
-        if constexpr (ARGMAX) { apart[pb * 32 + warp] = bestp; aidx[pb * 32 + warp] = bestq; }
-      }
-      __syncthreads();
-      if (tid == 0) {
-        float s0 = 0.f, s1 = 0.f;
+        __syncthreads();
+        if (tid == 0) {
+          float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-        for (int w2 = 0; w2 < nwarps; ++w2) { s0 += part[(pb * 32 + w2) * NP]; s1 += part[(pb * 32 + w2) * NP + 1]; }
-        if (P.out_soft) P.out_soft[seq * P.len + t] = s0 / (s1 * P.sk);
-        if constexpr (ARGMAX) {
-          float bp = -1.f;
-          int bq = 0x7fffffff;
+          for (int w2 = 0; w2 < nwarps; ++w2) { s0 += part[(pb * 32 + w2) * NP]; s1 += part[(pb * 32 + w2) * NP + 1]; }
+          if (P.out_soft) P.out_soft[seq * P.len + t] = s0 / (s1 * P.sk);
+          if constexpr (ARGMAX) {
+            float bp = -1.f;
+            int bq = 0x7fffffff;
 #pragma unroll
-          for (int w2 = 0; w2 < nwarps; ++w2) arg_better(bp, bq, apart[pb * 32 + w2], aidx[pb * 32 + w2]);
-          if (P.out_argmax) P.out_argmax[seq * n + t] = bq;
+            for (int w2 = 0; w2 < nwarps; ++w2) arg_better(bp, bq, apart[pb * 32 + w2], aidx[pb * 32 + w2]);
+            if (P.out_argmax) P.out_argmax[seq * n + t] = bq;
+          }
         }
       }
-      Cr -= (double)Rrn;
-      Rrn = bfly16_min(wmin[pb * 32 + (lane & 15)]);
+    } else {
+      float Rrn = 0.f;
+      double Cr = 0.0;   // log2 beta_t = -stored + Cr_t
+      float4 hsn = hist_in(hist, n - 1, tid);
+      for (int t = n - 1; t >= 0; --t) {
+        if (warp == 0) prefetch_history(hist, t, lane);
+        const float* ncur = lb[t & 1];
+        float* nnext = lb[(t + 1) & 1];
+        const float2 nw2 = f2s(wsc[t]);
+        const double Csig = (t >= 1) ? hist_c[t - 1] : 0.0;
+        const float K = (float)(Csig + Cr - l2Z);
+        const bool last = (t == n - 1);
+        float2 accc = f2s(0.f), accp = f2s(0.f);
+        float bestp = -1.f;
+        int bestq = 0x7fffffff;
+        float tmin = INFINITY;
+#pragma unroll
+        for (int k = 0; k < KB; ++k) {
+          const int mid = tid + NT * k;
+          float cb[16];
+          tmem_ld16(tbase + 16 * k, cb);
+          const float hs[4] = {hsn.x, hsn.y, hsn.z, hsn.w};
+          if (k + 1 < KB) hsn = hist_in(hist, t, mid + NT);
+          else if (t >= 1) hsn = hist_in(hist, t - 1, tid);
+          float nr[4];
+          if (last) {
+            nr[0] = nr[1] = nr[2] = nr[3] = 0.f;
+          } else {
+            const float4 rv = reinterpret_cast<const float4*>(ncur)[mid];
+            nr[0] = rv.x; nr[1] = rv.y; nr[2] = rv.z; nr[3] = rv.w;
+          }
+          float nout[4];
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {          // groups h = 2g, 2g+1 side by side
+            float2 y[4];
+#pragma unroll
+            for (int lo = 0; lo < 4; ++lo) {
+              const float2 d = __fadd2_rn(f2(cb[bidx(2 * g, lo)], cb[bidx(2 * g + 1, lo)]), nw2);
+              y[lo] = __ffma2_rn(d, d, f2s(nr[lo]));
+            }
+            // the posterior directly, p = 2^(K - n_sigma - y'), one ex2 per state
+            const float2 kh = __fadd2_rn(f2s(K), f2(-hs[2 * g], -hs[2 * g + 1]));
+            float2 ssum = f2s(0.f);
+#pragma unroll
+            for (int lo = 0; lo < 4; ++lo) {
+              const float2 a = __ffma2_rn(y[lo], neg1, kh);
+              const float2 pp = f2(ex2f(a.x), ex2f(a.y));
+              ssum = __fadd2_rn(ssum, pp);
+              accc = __ffma2_rn(pp, f2(cb[bidx(2 * g, lo)], cb[bidx(2 * g + 1, lo)]), accc);
+              if constexpr (ARGMAX) {
+                arg_better(bestp, bestq, pp.x, ((2 * g) << 14) | (mid << 2) | lo);
+                arg_better(bestp, bestq, pp.y, ((2 * g + 1) << 14) | (mid << 2) | lo);
+              }
+            }
+            accp = __fadd2_rn(accp, ssum);
+            // negated log rho_{t-1} = (K - n_sigma) - lg2 sum p (+inf, i.e. rho = 0, when the
+            // group's posterior mass underflows; it then moves no posterior by more than that mass)
+            nout[2 * g] = (kh.x - Rrn) - lg2f(ssum.x);
+            nout[2 * g + 1] = (kh.y - Rrn) - lg2f(ssum.y);
+          }
+          if (t >= 1) {
+#pragma unroll
+            for (int h = 0; h < 4; ++h) nnext[(h << HB) | mid] = nout[h];
+            tmin = fminf(tmin, fminf(fminf(nout[0], nout[1]), fminf(nout[2], nout[3])));
+          }
+        }
+        float a0 = warp_sum(accc.x + accc.y);
+        float a1 = warp_sum(accp.x + accp.y);
+        tmin = -warp_max(-tmin);
+        if constexpr (ARGMAX) warp_argmax(bestp, bestq);
+        const int pb = t & 1;
+        if (lane == 0) {
+          part[(pb * 32 + warp) * NP] = a0;
+          part[(pb * 32 + warp) * NP + 1] = a1;
+          wmin[pb * 32 + warp] = tmin;
+          if constexpr (ARGMAX) { apart[pb * 32 + warp] = bestp; aidx[pb * 32 + warp] = bestq; }
+        }
+        __syncthreads();
+        if (tid == 0) {
+          float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+          for (int w2 = 0; w2 < nwarps; ++w2) { s0 += part[(pb * 32 + w2) * NP]; s1 += part[(pb * 32 + w2) * NP + 1]; }
+          if (P.out_soft) P.out_soft[seq * P.len + t] = s0 / (s1 * P.sk);
+          if constexpr (ARGMAX) {
+            float bp = -1.f;
+            int bq = 0x7fffffff;
+#pragma unroll
+            for (int w2 = 0; w2 < nwarps; ++w2) arg_better(bp, bq, apart[pb * 32 + w2], aidx[pb * 32 + w2]);
+            if (P.out_argmax) P.out_argmax[seq * n + t] = bq;
+          }
+        }
+        Cr -= (double)Rrn;
+        Rrn = bfly16_min(wmin[pb * 32 + (lane & 15)]);
+      }
     }
     __syncthreads();
   }
@@ -406,24 +530,35 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
   if (warp == 0) tmem_dealloc512(tslot[0]);
 }
 
-
 // ------------------------------------------------------------ VJP pass, packed
 // Forward (negated log sigma and the prefix expectation A), then backward
-// (negated log rho, suffix expectation Bc, G, dl/dw per step and the per-state
-// codebook gradient).  Tensor memory holds the codewords during the forward
-// and the current sequence's codebook gradient during the backward, when the
-// codewords stream from L2 (block-major lines, prefetched one block ahead).
-// The forward's A_t ping-pongs in global scratch (L2-resident); both
-// histories (negated log sigma and A) go to HBM in block-major order [mid][h],
-// written by the next forward step from the values it has just read, so that
-// the backward loads one 16-byte vector of each per block.  The backward's Bc
-// ping-pongs in the same global scratch.
+// (suffix expectation, G, dl/dw per step and the per-state codebook gradient).
+// Tensor memory holds the codewords during the forward and the current
+// sequence's codebook gradient during the backward, when the codewords stream
+// from L2 (block-major lines, prefetched two units ahead).  The forward's A_t
+// ping-pongs in global scratch (L2-resident); the histories go to HBM: the
+// forward values in group order [t][j] (as in the soft pass) and A in
+// block-major order [mid][h], written by the next forward step from the values
+// it has just read, so that the backward loads one 16-byte vector per block
+// (the log-domain backward takes the forward values in that order too).
+//
+// Backward in posterior space (POST): with u_t(q) and P_t(j) as in the soft
+// pass and Bc_t the suffix expectation, the exchanged values are P_t(j) and
+// W_t(j) = P_t(j) (Bc_t(j) - Q_t) (Q_t a running reference), so that
+//     p_t(q) Bc-part = u_t(q) W_t(q mod J),
+//     W_{t-1}(i) = sum_lo [ p_t(q) (h_t(q) - rB_t) + u_t(q) W_t(q mod J) ],
+//     G_t(q) = p_t(q) (A_{t-1}(q >> 2) - K_t + gZ + h_t(q)) + u_t(q) W_t(q mod J),
+// with no logarithm and no division per group.  The log-domain backward
+// exchanges the negated log rho and Bc = W / P instead.  Both renormalise the
+// posterior mass of every step (its sum drifts from 1 by the rounding of the
+// two sweeps).
+template <bool POST>
 __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n = P.n;
 
   extern __shared__ __align__(16) float smem[];
-  float* sb = smem;                                    // [2][J] negated state ping-pong
+  float* sb = smem;                                    // [2][J] forward values / P or negated log rho
   float* lb[2] = {sb, sb + J};
   // per-warp partials of a step, [2 parities][32][8]:
   //   0: sum P(i) (A + Bc)   1: sum P(i) Bc   2: sum P(i)   3: min stored value
@@ -436,6 +571,7 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
   float* hist_l = P.hist_l + (size_t)blockIdx.x * n * J;
   float* hist_a = P.hist_a + (size_t)blockIdx.x * n * J;
   double* hist_c = P.hist_c + (size_t)blockIdx.x * n;
+  float* hist_rn = P.hist_rn + (size_t)blockIdx.x * n;
   float* bcg[2] = {P.bc_g + (size_t)blockIdx.x * 2 * J, P.bc_g + (size_t)blockIdx.x * 2 * J + J};
   double* gcp = P.gc_part + (size_t)blockIdx.x * S;
   const float* __restrict__ cs_tm = P.cs_tm;
@@ -503,7 +639,9 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
           np01 = f2(nprev[(0 << HB) | mid], nprev[(1 << HB) | mid]);
           np23 = f2(nprev[(2 << HB) | mid], nprev[(3 << HB) | mid]);
           // step t-1's values in block-major order [mid][h], as the backward reads them
-          reinterpret_cast<float4*>(hist_l + (size_t)(t - 1) * J)[mid] = make_float4(np01.x, np01.y, np23.x, np23.y);
+          // (the posterior space backward takes the forward values in group order instead)
+          if constexpr (!POST)
+            reinterpret_cast<float4*>(hist_l + (size_t)(t - 1) * J)[mid] = make_float4(np01.x, np01.y, np23.x, np23.y);
           reinterpret_cast<float4*>(hist_a + (size_t)(t - 1) * J)[mid] = make_float4(ap01.x, ap01.y, ap23.x, ap23.y);
         }
         float out[4], aout[4];
@@ -523,20 +661,23 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
           aout[lo] = __fdividef(q2.x + q2.y, ssum);
         }
         tmin = fminf(tmin, fminf(fminf(out[0], out[1]), fminf(out[2], out[3])));
-        reinterpret_cast<float4*>(ncur)[mid] = make_float4(out[0], out[1], out[2], out[3]);
+        const float4 ov = make_float4(out[0], out[1], out[2], out[3]);
+        reinterpret_cast<float4*>(ncur)[mid] = ov;
+        if constexpr (POST) reinterpret_cast<float4*>(hist_l + (size_t)t * J)[mid] = ov;
         reinterpret_cast<float4*>(acur)[mid] = make_float4(aout[0], aout[1], aout[2], aout[3]);
       }
       tmin = -warp_max(-tmin);
       if (lane == 0) rec[((t & 1) * 32 + warp) * 8 + 3] = tmin;
-      if (tid == 0) hist_c[t] = C;
+      if (tid == 0) { hist_c[t] = C; hist_rn[t] = Rn; }
       __syncthreads();
       Rn = bfly16_min(rec[((t & 1) * 32 + (lane & 15)) * 8 + 3]);
     }
-    // log2 Z and Hbar = E[A_{n-1}]
+    // log2 Z and Hbar = E[A_{n-1}]; the posterior space backward starts from
+    // P_{n-1}(j) = 2^(Rn - stored_j) / sum, written in place
     double l2Z;
     float Hbar;
     {
-      const float* nfin = lb[(n - 1) & 1];
+      float* nfin = lb[(n - 1) & 1];
       const float* afin = bcg[(n - 1) & 1];
       float s0 = 0.f, s1 = 0.f;
       for (int j = tid; j < J; j += NT) {
@@ -552,6 +693,10 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
       const float a1 = bfly16_sum(rec[(lane & 15) * 8 + 5]);
       l2Z = -(double)Rn + log2((double)a0) + C;
       Hbar = a1 / a0;
+      if constexpr (POST) {
+        const float inv = 1.f / a0;
+        for (int j = tid; j < J; j += NT) nfin[j] = ex2f(Rn - nfin[j]) * inv;
+      }
       __syncthreads();
     }
     const float gzq = P.gZ ? P.gZ[seq] : 0.f;
@@ -569,25 +714,39 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
 
     // ------------------------------------------------------------ backward
     // Work unit = one h-pair g of one block k: 8 states, 8 codewords, 8 TMEM
-    // columns; codewords and history values are prefetched one unit ahead.
-    float Rrn = 0.f;
-    double Cr = 0.0;
-    // G_t(q) = p_t(q) (A_{t-1}(q >> 2) + h_t(q) + Bc_t(q mod J) - K_t + gZ) with
-    // K_t = sum_j P_t(j) (A_t(j) + Bc_t(j)), P_t(j) the posterior of group j,
+    // columns; codewords are prefetched two units ahead, history values one block ahead.
+    // K_t = sum_j P_t(j) (A_t(j) + Bc_t(j)) (P_t(j) the posterior of group j) is
     // formed from the same stored values one step earlier (K_{n-1} = Hbar), so
     // that rounding carried along the recursions cancels in G.  Stored Bc_t is
     // relative to rB, the posterior mean of the previous step's stored values.
     float Kt = Hbar, rB = 0.f;
-    float cbn[8], cbm[8];
+    float cbn[8];
     ld_cb8(cs_tm, tid, 0, cbn);
+#if BCJR_VJP_CB_AHEAD == 2
+    float cbm[8];
     ld_cb8(cs_tm, tid, 1, cbm);
-    // block kk of step tt reads step tt-1's values (free start: 0 for tt = 0)
-    auto hist_at = [&](const float* hbuf, int tt, int kk) -> float4 {
-      return (tt >= 1) ? reinterpret_cast<const float4*>(hbuf + (size_t)(tt - 1) * J)[tid + NT * kk]
+#endif
+    // block kk of step tt: A of step tt-1 in block-major order (free start: 0 for tt = 0)
+    auto hist_a_at = [&](int tt, int kk) -> float4 {
+      return (tt >= 1) ? reinterpret_cast<const float4*>(hist_a + (size_t)(tt - 1) * J)[tid + NT * kk]
                        : make_float4(0.f, 0.f, 0.f, 0.f);
     };
-    float4 hsn = hist_at(hist_l, n - 1, 0), han = hist_at(hist_a, n - 1, 0);
+    // forward values of step tt-1 for block kk: four scalars of the group-order
+    // history (posterior space) or one vector of the block-major one (log domain)
+    auto hist_l_at = [&](int tt, int kk) -> float4 {
+      if constexpr (POST) return hist_in(hist_l, tt, tid + NT * kk);
+      return (tt >= 1) ? reinterpret_cast<const float4*>(hist_l + (size_t)(tt - 1) * J)[tid + NT * kk]
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    };
+    float4 hin_n = hist_l_at(n - 1, 0), han = hist_a_at(n - 1, 0);
+#if BCJR_VJP_HOUT_AHEAD
+    float4 hout_n = POST ? hist_out(hist_l, n - 1, tid) : make_float4(0.f, 0.f, 0.f, 0.f);
+#endif
+    float lsp = 0.f;     // log2 of the previous step's posterior mass (POST)
+    float Rrn = 0.f;     // log domain: min of the previous step's stored values
+    double Cr = 0.0;     // log domain: log2 beta_t = -stored + Cr_t
     for (int t = n - 1; t >= 0; --t) {
+      if (warp == 0) prefetch_history(hist_l, t, lane);
       const float* ncur = lb[t & 1];
       float* nnext = lb[(t + 1) & 1];
       const float* bcur = bcg[t & 1];
@@ -596,11 +755,14 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
       const float2 nw2 = f2s(nwt);
       const float2 g2 = f2s(gsc[t]);
       const float2 gr2 = f2s(gsc[t] * P.sk);
-      const double Csig = (t >= 1) ? hist_c[t - 1] : 0.0;
-      const float K = (float)(Csig + Cr - l2Z);
       const bool last = (t == n - 1);
       const float rA = (t >= 1) ? hist_a[(size_t)(t - 1) * J] : 0.f;   // the forward's reference
       const float hbt = Kt + rA - rB - gzq;
+      // POST: 2^(n_t + Rn_t - x) / (posterior mass); log domain: K = log2 of 1/Z and the offsets
+      const float nrs = POST ? hist_rn[t] - lsp : 0.f;
+      float K = 0.f;
+      if constexpr (!POST) K = (float)(((t >= 1) ? hist_c[t - 1] : 0.0) + Cr - l2Z);
+      const float2 nrB2 = f2s(-rB);
       float2 accGd = f2s(0.f);   // sum_q G (c' - w')
       float2 accK = f2s(0.f), accB = f2s(0.f), accP = f2s(0.f);
       float tmin = INFINITY;
@@ -609,75 +771,138 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
 #pragma unroll
       for (int k = 0; k < KB; ++k) {
         const int mid = tid + NT * k;
-        float nr[4], bc[4];
-        if (last) {
+        float nr[4], bc[4];   // P and W (POST) or negated log rho and Bc
+        if (last && !POST) {
           nr[0] = nr[1] = nr[2] = nr[3] = 0.f;
-          bc[0] = bc[1] = bc[2] = bc[3] = 0.f;
         } else {
           const float4 rv = reinterpret_cast<const float4*>(ncur)[mid];
           nr[0] = rv.x; nr[1] = rv.y; nr[2] = rv.z; nr[3] = rv.w;
-          bc[0] = bvn.x - rB; bc[1] = bvn.y - rB; bc[2] = bvn.z - rB; bc[3] = bvn.w - rB;
+        }
+        if (last) {
+          bc[0] = bc[1] = bc[2] = bc[3] = 0.f;
+        } else {
+          if constexpr (POST) {
+            bc[0] = bvn.x; bc[1] = bvn.y; bc[2] = bvn.z; bc[3] = bvn.w;
+          } else {
+            bc[0] = bvn.x - rB; bc[1] = bvn.y - rB; bc[2] = bvn.z - rB; bc[3] = bvn.w - rB;
+          }
         }
         if (!last && k + 1 < KB) bvn = reinterpret_cast<const float4*>(bcur)[mid + NT];
-        const float4 hs4 = hsn, ha4 = han;
-        {
-          const int nt = (k + 1 < KB) ? t : t - 1, nk = (k + 1 < KB) ? k + 1 : 0;
-          hsn = hist_at(hist_l, nt, nk);
-          han = hist_at(hist_a, nt, nk);
+#if BCJR_VJP_HOUT_AHEAD
+        const float4 hi4 = hin_n, ha4 = han, ho4 = hout_n;
+#else
+        const float4 hi4 = hin_n, ha4 = han;
+        const float4 ho4 = POST ? hist_out(hist_l, t, mid) : make_float4(0.f, 0.f, 0.f, 0.f);
+#endif
+        if (k + 1 < KB) {
+          hin_n = hist_l_at(t, k + 1);
+          han = hist_a_at(t, k + 1);
+#if BCJR_VJP_HOUT_AHEAD
+          if constexpr (POST) hout_n = hist_out(hist_l, t, mid + NT);
+#endif
+        } else if (t >= 1) {
+          hin_n = hist_l_at(t - 1, 0);
+          han = hist_a_at(t - 1, 0);
+#if BCJR_VJP_HOUT_AHEAD
+          if constexpr (POST) hout_n = hist_out(hist_l, t - 1, tid);
+#endif
+        }
+        float lnr[4];   // POST: n_t(j) + Rn_t - log2 mass
+        if constexpr (POST) {
+          lnr[0] = ho4.x + nrs; lnr[1] = ho4.y + nrs; lnr[2] = ho4.z + nrs; lnr[3] = ho4.w + nrs;
         }
         float nout[4], bout[4];
 #pragma unroll
         for (int g = 0; g < 2; ++g) {          // groups h = 2g, 2g+1 side by side
           float cb[8];
+#if BCJR_VJP_CB_AHEAD == 2
 #pragma unroll
           for (int i = 0; i < 8; ++i) { cb[i] = cbn[i]; cbn[i] = cbm[i]; }
-          const float hs0 = g ? hs4.z : hs4.x, hs1 = g ? hs4.w : hs4.y;
-          const float ha0 = g ? ha4.z : ha4.x, ha1 = g ? ha4.w : ha4.y;
           {
             // codewords two units after (k, g): block k+1 (or 0), same g
             const int nk = (k + 1 < KB) ? k + 1 : 0;
             ld_cb8(cs_tm, tid + NT * nk, g, cbm);
           }
+#else
+#pragma unroll
+          for (int i = 0; i < 8; ++i) cb[i] = cbn[i];
+          {
+            // codewords one unit after (k, g)
+            const int nk = g ? ((k + 1 < KB) ? k + 1 : 0) : k;
+            ld_cb8(cs_tm, tid + NT * nk, g ^ 1, cbn);
+          }
+#endif
+          const float hs0 = g ? hi4.z : hi4.x, hs1 = g ? hi4.w : hi4.y;
+          const float ha0 = g ? ha4.z : ha4.x, ha1 = g ? ha4.w : ha4.y;
           float gcb[8];
           tmem_ld8(tbase + 16 * k + 8 * g, gcb);
-          float2 y[4], c2[4];
+          const float2 ah = f2(ha0 - hbt, ha1 - hbt);   // A - K + gZ (+ rB in POST)
+          if constexpr (POST) {
+            const float2 np2 = f2(hs0, hs1);
+            float2 Pn = f2s(0.f), Wn = f2s(0.f);
 #pragma unroll
-          for (int lo = 0; lo < 4; ++lo) {
-            c2[lo] = f2(cb[2 * lo], cb[2 * lo + 1]);
-            const float2 dd = __fadd2_rn(c2[lo], nw2);
-            y[lo] = __ffma2_rn(dd, dd, f2s(nr[lo]));
-          }
-          // the posterior directly, p = 2^(K - n_sigma - y'), one ex2 per state
-          const float2 kh = __fadd2_rn(f2s(K), f2(-hs0, -hs1));
-          const float2 ah = f2(ha0 - hbt, ha1 - hbt);   // A - K + gZ
-          float2 ssum = f2s(0.f), num = f2s(0.f);
+            for (int lo = 0; lo < 4; ++lo) {
+              const float2 c2 = f2(cb[2 * lo], cb[2 * lo + 1]);
+              const float2 dd = __fadd2_rn(c2, nw2);
+              const float2 a = __ffma2_rn(__ffma2_rn(dd, dd, np2), neg1, f2s(lnr[lo]));
+              const float2 u = f2(ex2f(a.x), ex2f(a.y));
+              const float2 pp = __fmul2_rn(u, f2s(nr[lo]));           // posterior
+              const float2 uw = __fmul2_rn(u, f2s(bc[lo]));           // u W
+              const float2 v = __ffma2_rn(pp, __ffma2_rn(g2, c2, nrB2), uw);   // p (h - rB) + u W
+              const float2 G = __ffma2_rn(pp, ah, v);
+              Pn = __fadd2_rn(Pn, pp);
+              Wn = __fadd2_rn(Wn, v);
+              const float2 Gd = __fmul2_rn(G, dd);                    // G (c' - w')
+              accGd = __fadd2_rn(accGd, Gd);
+              float2 gc = f2(gcb[2 * lo], gcb[2 * lo + 1]);
+              gc = __ffma2_rn(Gd, nc2T, __ffma2_rn(gr2, pp, gc));    // + g p + (2/T) G (w - c)
+              gcb[2 * lo] = gc.x;
+              gcb[2 * lo + 1] = gc.y;
+            }
+            nout[2 * g] = Pn.x; nout[2 * g + 1] = Pn.y;
+            bout[2 * g] = Wn.x; bout[2 * g + 1] = Wn.y;
+            accK = __ffma2_rn(Pn, f2(ha0, ha1), __fadd2_rn(accK, Wn));
+            accB = __fadd2_rn(accB, Wn);
+            accP = __fadd2_rn(accP, Pn);
+          } else {
+            float2 y[4], c2[4];
 #pragma unroll
-          for (int lo = 0; lo < 4; ++lo) {
-            const float2 a = __ffma2_rn(y[lo], neg1, kh);
-            const float2 pp = f2(ex2f(a.x), ex2f(a.y));
-            ssum = __fadd2_rn(ssum, pp);
-            const float2 z = __ffma2_rn(g2, c2[lo], f2s(bc[lo]));          // Bc + h
-            num = __ffma2_rn(pp, z, num);
-            const float2 G = __fmul2_rn(pp, __fadd2_rn(z, ah));
-            const float2 Gd = __fmul2_rn(G, __fadd2_rn(c2[lo], nw2));   // G (c' - w')
-            accGd = __fadd2_rn(accGd, Gd);
-            float2 gc = f2(gcb[2 * lo], gcb[2 * lo + 1]);
-            gc = __ffma2_rn(Gd, nc2T, __ffma2_rn(gr2, pp, gc));       // + g p + (2/T) G (w - c)
-            gcb[2 * lo] = gc.x;
-            gcb[2 * lo + 1] = gc.y;
+            for (int lo = 0; lo < 4; ++lo) {
+              c2[lo] = f2(cb[2 * lo], cb[2 * lo + 1]);
+              const float2 dd = __fadd2_rn(c2[lo], nw2);
+              y[lo] = __ffma2_rn(dd, dd, f2s(nr[lo]));
+            }
+            // the posterior directly, p = 2^(K - n_sigma - y'), one ex2 per state
+            const float2 kh = __fadd2_rn(f2s(K), f2(-hs0, -hs1));
+            float2 ssum = f2s(0.f), num = f2s(0.f);
+#pragma unroll
+            for (int lo = 0; lo < 4; ++lo) {
+              const float2 a = __ffma2_rn(y[lo], neg1, kh);
+              const float2 pp = f2(ex2f(a.x), ex2f(a.y));
+              ssum = __fadd2_rn(ssum, pp);
+              const float2 z = __ffma2_rn(g2, c2[lo], f2s(bc[lo]));          // Bc + h
+              num = __ffma2_rn(pp, z, num);
+              const float2 G = __fmul2_rn(pp, __fadd2_rn(z, ah));
+              const float2 Gd = __fmul2_rn(G, __fadd2_rn(c2[lo], nw2));   // G (c' - w')
+              accGd = __fadd2_rn(accGd, Gd);
+              float2 gc = f2(gcb[2 * lo], gcb[2 * lo + 1]);
+              gc = __ffma2_rn(Gd, nc2T, __ffma2_rn(gr2, pp, gc));       // + g p + (2/T) G (w - c)
+              gcb[2 * lo] = gc.x;
+              gcb[2 * lo + 1] = gc.y;
+            }
+            // negated log rho_{t-1} = (K - n_sigma) - lg2 sum p; a group whose posterior mass
+            // underflows gets rho = 0 (+inf) and Bc = 0, moving no posterior by more than that mass
+            nout[2 * g] = (kh.x - Rrn) - lg2f(ssum.x);
+            nout[2 * g + 1] = (kh.y - Rrn) - lg2f(ssum.y);
+            bout[2 * g] = (ssum.x > 0.f) ? __fdividef(num.x, ssum.x) : 0.f;
+            bout[2 * g + 1] = (ssum.y > 0.f) ? __fdividef(num.y, ssum.y) : 0.f;
+            // posterior of the two step t-1 groups, P(i) = sum_lo p
+            const float2 pg = ssum, bo = f2(bout[2 * g], bout[2 * g + 1]);
+            accK = __ffma2_rn(pg, __fadd2_rn(f2(ha0, ha1), bo), accK);
+            accB = __ffma2_rn(pg, bo, accB);
+            accP = __fadd2_rn(accP, pg);
           }
           tmem_st8(tbase + 16 * k + 8 * g, gcb);
-          // negated log rho_{t-1} = (K - n_sigma) - lg2 sum p; a group whose posterior mass
-          // underflows gets rho = 0 (+inf) and Bc = 0, moving no posterior by more than that mass
-          nout[2 * g] = (kh.x - Rrn) - lg2f(ssum.x);
-          nout[2 * g + 1] = (kh.y - Rrn) - lg2f(ssum.y);
-          bout[2 * g] = (ssum.x > 0.f) ? __fdividef(num.x, ssum.x) : 0.f;
-          bout[2 * g + 1] = (ssum.y > 0.f) ? __fdividef(num.y, ssum.y) : 0.f;
-          // posterior of the two step t-1 groups, P(i) = sum_lo p
-          const float2 pg = ssum, bo = f2(bout[2 * g], bout[2 * g + 1]);
-          accK = __ffma2_rn(pg, __fadd2_rn(f2(ha0, ha1), bo), accK);
-          accB = __ffma2_rn(pg, bo, accB);
-          accP = __fadd2_rn(accP, pg);
         }
         if (t >= 1) {
 #pragma unroll
@@ -685,7 +910,7 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
             nnext[(h << HB) | mid] = nout[h];
             bnext[(h << HB) | mid] = bout[h];
           }
-          tmin = fminf(tmin, fminf(fminf(nout[0], nout[1]), fminf(nout[2], nout[3])));
+          if constexpr (!POST) tmin = fminf(tmin, fminf(fminf(nout[0], nout[1]), fminf(nout[2], nout[3])));
         }
       }
       tmem_wait_st();
@@ -693,7 +918,7 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
       const float kk = warp_sum(accK.x + accK.y);
       const float kb = warp_sum(accB.x + accB.y);
       const float kp = warp_sum(accP.x + accP.y);
-      tmin = -warp_max(-tmin);
+      if constexpr (!POST) tmin = -warp_max(-tmin);
       const int pb = t & 1;
       if (lane == 0) {
         float* r = rec + (pb * 32 + warp) * 8;
@@ -708,17 +933,21 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
         // dl/dw_t = (2/T) sum_q G (c - w_t) = (2/T) sum_q G (c' - w') / sk
         P.grad_w[seq * P.len + t] = P.two_over_T * s0 / P.sk;
       }
-      Cr -= (double)Rrn;
       {
         const float4 r = *reinterpret_cast<const float4*>(rec + (pb * 32 + (lane & 15)) * 8);
         const float sp = bfly16_sum(r.z);   // sum_q p_t(q), 1 up to rounding
         Kt = bfly16_sum(r.x) / sp;
         rB = bfly16_sum(r.y) / sp;
-        Rrn = bfly16_min(r.w);
-        // Forward and backward carry different rounding relative to the one
-        // log Z, so the posterior sum drifts from 1 along the sweep; folding
-        // its logarithm into the backward offset renormalises every next step.
-        Cr -= (double)lg2f(sp);
+        // Forward and backward carry different rounding, so the posterior sum
+        // drifts from 1 along the sweep; dividing it out renormalises every
+        // next step.
+        if constexpr (POST) {
+          lsp = lg2f(sp);
+        } else {
+          Cr -= (double)Rrn;
+          Rrn = bfly16_min(r.w);
+          Cr -= (double)lg2f(sp);
+        }
       }
     }
 
@@ -740,7 +969,6 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
   tmem_fence_after();
   if (warp == 0) tmem_dealloc512(tslot[0]);
 }
-
 
 // ------------------------------------------------------------ Viterbi
 // The T -> 0 decode in the same block layout: per step and forward group
