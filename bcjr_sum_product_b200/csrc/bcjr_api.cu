@@ -133,14 +133,18 @@ int threads_for(int J, int B) {
   return (t + 31) / 32 * 32;
 }
 
+// Resident CTAs of `kernel` over the device (at most n_seq).  A failed query
+// clears the CUDA error it leaves, so that it is not reported by a later call.
 template <class K>
 int grid_for(K kernel, int threads, size_t smem, int64_t n_seq, int* grid) {
   int dev = 0, nsm = 0, per = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return BCJR_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return BCJR_ERR_CUDA;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kernel, threads, smem) != cudaSuccess) {
+    cudaGetLastError();
     return BCJR_ERR_CUDA;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kernel, threads, smem) != cudaSuccess) return BCJR_ERR_CUDA;
+  }
   if (per < 1) return BCJR_ERR_UNSUPPORTED;
   int64_t g = (int64_t)per * nsm;
   if (g > n_seq) g = n_seq;
@@ -525,7 +529,8 @@ int run_viterbi(const Shape& sh, const float* w, const float* c, int32_t* out_st
   return BCJR_OK;
 }
 
-static_assert(bcjr::kErrTimeout == BCJR_ERR_TIMEOUT, "device and host status codes agree");
+static_assert(bcjr::kErrTimeout == BCJR_ERR_TIMEOUT && bcjr::kErrNumeric == BCJR_ERR_NUMERIC,
+              "device and host status codes agree");
 
 }  // namespace
 
@@ -650,6 +655,7 @@ const char* bcjr_strerror(int status) {
     case BCJR_ERR_UNSUPPORTED: return "unsupported configuration";
     case BCJR_ERR_CUDA: return "CUDA error";
     case BCJR_ERR_TIMEOUT: return "device-side wait timed out";
+    case BCJR_ERR_NUMERIC: return "numerical check failed on the device (posterior mass off)";
     default: return "unknown status";
   }
 }
@@ -715,6 +721,7 @@ extern "C" int bcjr_soft_codeword_noalloc(const float* w, int64_t n_seq, int64_t
   const size_t state_bytes = sizeof(float) * (size_t)sh.J * 2;
   const bool in_smem = fixed + state_bytes <= kMaxDynSmem;
   const size_t smem = fixed + (in_smem ? state_bytes : 0);
+  if (smem > kMaxDynSmem) return BCJR_ERR_UNSUPPORTED;
   int grid = 0;
   if ((rc = grid_for(kern, threads, smem, sh.n_seq, &grid))) return rc;
 
@@ -729,13 +736,24 @@ extern "C" int bcjr_soft_codeword_noalloc(const float* w, int64_t n_seq, int64_t
     P.gc_seq = nullptr;
     P.gc_part = nullptr;
   };
-  // Fewer CTAs when the fixed scratch cannot hold one history per resident CTA.
-  for (;;) {
+  // As many CTAs as the fixed array holds histories for: the codebook and each
+  // of the three per-CTA arrays take at most 255 bytes of alignment padding.
+  {
+    const size_t cb = (sizeof(float) * SV + 255) & ~size_t(255);
+    const size_t per_cta = sizeof(float) * (size_t)sh.n * sh.J + sizeof(double) * sh.n +
+                           (in_smem ? 0 : sizeof(float) * 4 * (size_t)sh.J);
+    const size_t cap = BCJR_NOALLOC_SCRATCH_BYTES;
+    if (cb + 3 * 256 + per_cta > cap) return BCJR_ERR_UNSUPPORTED;   // one sequence does not fit
+    const size_t fit = (cap - cb - 3 * 256) / per_cta;
+    if ((size_t)grid > fit) grid = (int)fit;
     Arena sizing;
     layout(sizing, grid);
-    if (sizing.off <= (size_t)BCJR_NOALLOC_SCRATCH_BYTES) break;
-    if (grid == 1) return BCJR_ERR_UNSUPPORTED;  // one sequence's scratch exceeds the array
-    grid = grid / 2 > 0 ? grid / 2 : 1;
+    while (sizing.off > cap && grid > 1) {   // the padding bound above makes this a no-op
+      --grid;
+      sizing = Arena{};
+      layout(sizing, grid);
+    }
+    if (sizing.off > cap) return BCJR_ERR_UNSUPPORTED;
   }
   void* base = nullptr;
   if ((rc = noalloc_scratch(&base))) return rc;
@@ -753,3 +771,4 @@ extern "C" int bcjr_soft_codeword_noalloc(const float* w, int64_t n_seq, int64_t
   kern<<<grid, threads, smem, st>>>(P);
   return cudaGetLastError() == cudaSuccess ? BCJR_OK : BCJR_ERR_CUDA;
 }
+

@@ -42,8 +42,16 @@ constexpr int kMaxWarps = kMaxThreads / 32;
 // First device-side error recorded by a kernel of this library (a status code
 // of the C interface, 0 = none); read and cleared by bcjr_get_device_error.
 __device__ int g_device_error = 0;
-constexpr int kErrTimeout = 4;   // a bounded wait ran out
+constexpr int kErrTimeout = 4;   // reserved: no kernel of this version waits on a flag
+constexpr int kErrNumeric = 5;   // a per-step posterior mass left 1 +- 1e-2, or was not finite
 __device__ __forceinline__ void record_device_error(int code) { atomicCAS(&g_device_error, 0, code); }
+// The posterior of every step sums to 1 (both sweeps are exact rewritings of
+// the same marginals); a sum off by more than 1e-2 (rounding keeps it within
+// about 1e-4 even at T = 0.01 and 8192 steps) or not finite (NaN or infinite
+// inputs) means the sequence's outputs are not usable.
+__device__ __forceinline__ void check_posterior_mass(float s) {
+  if (!(fabsf(s - 1.f) <= 1e-2f)) record_device_error(kErrNumeric);
+}
 
 struct SweepParams {
   const float* w;        // [n_seq][len]
@@ -390,6 +398,7 @@ __global__ void __launch_bounds__(kMaxThreads) bcjr_sweep_kernel(SweepParams P) 
           tot[k2] = a;
         }
         if constexpr (MODE == MODE_SOFT) {
+          check_posterior_mass(tot[V]);
           if (P.out_soft) {
             const float inv = 1.f / (tot[V] * P.sk);
 #pragma unroll
@@ -418,6 +427,8 @@ __global__ void __launch_bounds__(kMaxThreads) bcjr_sweep_kernel(SweepParams P) 
         }
         Kt = sk_ / sp_;
         rB = sb_ / sp_;
+        // (step 0 has no predecessor groups, so no mass is summed there)
+        if (tid == 0 && t >= 1) check_posterior_mass(sp_);
         // sp_ = sum_q p_t(q): forward and backward carry different rounding
         // relative to the one log Z, so the posterior sum drifts from 1 along
         // the sweep; folding its logarithm into the backward offset

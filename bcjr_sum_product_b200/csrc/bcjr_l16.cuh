@@ -416,6 +416,7 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
           float s0 = 0.f, s1 = 0.f;
 #pragma unroll
           for (int w2 = 0; w2 < nwarps; ++w2) { s0 += part[(pb * 32 + w2) * NP]; s1 += part[(pb * 32 + w2) * NP + 1]; }
+          check_posterior_mass(s1);
           if (P.out_soft) P.out_soft[seq * P.len + t] = s0 / (s1 * P.sk);
           if constexpr (ARGMAX) {
             float bp = -1.f;
@@ -508,6 +509,7 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
           float s0 = 0.f, s1 = 0.f;
 #pragma unroll
           for (int w2 = 0; w2 < nwarps; ++w2) { s0 += part[(pb * 32 + w2) * NP]; s1 += part[(pb * 32 + w2) * NP + 1]; }
+          check_posterior_mass(s1);
           if (P.out_soft) P.out_soft[seq * P.len + t] = s0 / (s1 * P.sk);
           if constexpr (ARGMAX) {
             float bp = -1.f;
@@ -938,6 +940,7 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
         const float sp = bfly16_sum(r.z);   // sum_q p_t(q), 1 up to rounding
         Kt = bfly16_sum(r.x) / sp;
         rB = bfly16_sum(r.y) / sp;
+        if (tid == 0) check_posterior_mass(sp);
         // Forward and backward carry different rounding, so the posterior sum
         // drifts from 1 along the sweep; dividing it out renormalises every
         // next step.

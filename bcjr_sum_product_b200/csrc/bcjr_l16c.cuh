@@ -458,6 +458,7 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
         const float sp = bfly32_sum(rv.z);   // sum_q p_t(q), 1 up to rounding
         Kt = bfly32_sum(rv.x) / sp;
         rB = bfly32_sum(rv.y) / sp;
+        if (r == 0 && tid == 0) check_posterior_mass(sp);
         Rrn = bfly32_min(rv.w);
         // Forward and backward carry different rounding relative to the one
         // log Z, so the posterior sum drifts from 1 along the sweep; folding

@@ -318,6 +318,7 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
           const float* r = rec + (pb * 32 + w2) * 8;
           s0 += r[1]; s1 += r[2]; s2 += r[3];
         }
+        check_posterior_mass(s2);
         if (P.out_soft) {
           const float inv = 1.f / (s2 * P.sk);
           P.out_soft[seq * P.len + 2 * t] = s0 * inv;
@@ -624,6 +625,7 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
         const float sp = bfly16_sum(r.z);   // sum_q p_t(q), 1 up to rounding
         Kt = bfly16_sum(r.x) / sp;
         rB = bfly16_sum(r.y) / sp;
+        if (tid == 0) check_posterior_mass(sp);
         Rrn = bfly16_min(r.w);
         // renormalise the next step's posterior (the drift of the posterior sum)
         Cr -= (double)lg2f(sp);

@@ -21,6 +21,7 @@ BCJR_ERR_INVALID_ARG = 1
 BCJR_ERR_UNSUPPORTED = 2
 BCJR_ERR_CUDA = 3
 BCJR_ERR_TIMEOUT = 4
+BCJR_ERR_NUMERIC = 5
 
 EXPORTS = ("bcjr_soft_codeword", "bcjr_vjp", "viterbi_decode", "bcjr_posterior_argmax",
            "bcjr_get_device_error", "bcjr_strerror", "bcjr_version")
@@ -59,7 +60,7 @@ def load(path: str = LIB_PATH):
             lib.bcjr_version.argtypes = []
             lib.bcjr_version.restype = ctypes.c_char_p
             for name in ("bcjr_soft_codeword", "bcjr_vjp", "viterbi_decode", "bcjr_posterior_argmax",
-                         "bcjr_get_device_error"):
+                         "bcjr_qat_step", "bcjr_get_device_error"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
     return _lib

@@ -44,7 +44,10 @@
  *     L > 16, D > 6, V not in {1,2,4}, len > 8192 -> BCJR_ERR_UNSUPPORTED;
  *     a failed CUDA call (allocation, launch)   -> BCJR_ERR_CUDA.
  *   - NaN or infinite weights make that sequence's outputs NaN; other
- *     sequences are unaffected.
+ *     sequences are unaffected.  The soft-codeword and VJP kernels also check
+ *     that the posterior of every step sums to 1 within 1e-2 and, if not (NaN
+ *     or infinite inputs, or a numerical breakdown), record BCJR_ERR_NUMERIC
+ *     for bcjr_get_device_error.
  */
 #ifndef BCJR_H_
 #define BCJR_H_
@@ -66,7 +69,8 @@ typedef enum {
   BCJR_ERR_INVALID_ARG = 1,
   BCJR_ERR_UNSUPPORTED = 2,
   BCJR_ERR_CUDA = 3,
-  BCJR_ERR_TIMEOUT = 4
+  BCJR_ERR_TIMEOUT = 4,  /* reserved: no kernel of this version waits on a flag */
+  BCJR_ERR_NUMERIC = 5   /* recorded on the device: a step's posterior mass was off */
 } bcjr_status;
 
 /*
@@ -128,7 +132,12 @@ BCJR_API int bcjr_posterior_argmax(const float* w, int64_t n_seq, int64_t len, i
  * latency-critical path where an allocation could block or fail under memory
  * pressure.
  *
- * Arguments, layouts, results and errors are those of bcjr_soft_codeword.
+ * Arguments, layouts and errors are those of bcjr_soft_codeword, and so are
+ * the results up to rounding: this entry point always runs the general sweep
+ * kernel, also where bcjr_soft_codeword runs a specialised one (L = 16 with
+ * k*V = 2 or 4), so the two agree within the soft-codeword and logZ
+ * tolerances (1e-5 of max|c| and of max(|logZ|, (L + D(n-1)) ln 2)), not bit
+ * for bit.
  * The call makes no cudaMalloc, cudaMallocAsync or cudaFree call and uses no
  * allocating library routine.  Its scratch space is one fixed array of
  * BCJR_NOALLOC_SCRATCH_BYTES (64 MiB) in this library's device memory; every
@@ -142,8 +151,11 @@ BCJR_API int bcjr_posterior_argmax(const float* w, int64_t n_seq, int64_t len, i
  * sequences run concurrently: slower, same results.
  *
  * Set-up: the first call on each device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture on the device.
+ * (cudaGetSymbolAddress, with that device current) and keeps it for the rest
+ * of the process; make that first call before any stream capture on the
+ * device.  A cudaDeviceReset (or any other way of unloading the library's
+ * module from the device) makes the kept address stale: do not call this entry
+ * point on a device after resetting it.
  *
  * Sharing: all calls on a device use the same array, which keeps whatever the
  * last call left in it (nothing in it needs to start at zero).  Calls whose
@@ -186,8 +198,9 @@ BCJR_API int bcjr_qat_step(float* w, const float* w_target, int64_t n_seq, int64
 /*
  * Synchronises `stream` and returns BCJR_OK, or BCJR_ERR_CUDA if the stream
  * holds a CUDA error, or the first device-side error recorded by a kernel of
- * this library since the last call (BCJR_ERR_TIMEOUT for a bounded wait that
- * ran out).  Reading the flag clears it.
+ * this library since the last call (BCJR_ERR_NUMERIC: a step's posterior mass
+ * left 1 +- 1e-2 or was not finite).  The flag is one per device and process,
+ * shared by all streams; reading it clears it.
  */
 BCJR_API int bcjr_get_device_error(void* stream);
 

@@ -41,6 +41,7 @@ def test_strerror_strings():
     assert lib.strerror(0) == "ok"
     assert "invalid" in lib.strerror(1)
     assert "unsupported" in lib.strerror(2)
+    assert "numerical" in lib.strerror(5)
     assert lib.strerror(99) == "unknown status"
 
 

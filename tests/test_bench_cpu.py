@@ -24,6 +24,22 @@ def test_reference_arm_prints_one_contract_line():
     assert d["config"]["workload"].startswith("tiny:")
 
 
+def test_reference_arm_viterbi_mode():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--viterbi",
+                          "--workload", "tiny", "--steps", "1", "--warmup", "0"],
+                         capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    d = json.loads(out.stdout.strip().splitlines()[-1])
+    assert d["impl"] == "reference" and d["value"] > 0 and "Viterbi" in d["metric"]
+    assert "Viterbi decode" in d["config"]["workload"] and d["dtype"] == "f32"
+
+
+def test_qat_and_viterbi_modes_exclude_each_other():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--qat", "--viterbi"],
+                         capture_output=True, text=True, timeout=120, cwd=ROOT)
+    assert out.returncode != 0 and "not allowed" in out.stderr
+
+
 def test_bad_temperature_is_rejected():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--workload", "mlp", "--temp", "0.5"],
                          capture_output=True, text=True, timeout=120, cwd=ROOT)

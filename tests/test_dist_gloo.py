@@ -44,6 +44,70 @@ def _worker(rank, world, port, out_dir):
     dist.destroy_process_group()
 
 
+def _bench_worker(rank, world, port, out_dir, replicate):
+    """bench.py's own multi-rank step (its row split and its two halves), with
+    the CPU oracle as the local soft codeword and VJP."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    import bench
+    import oracle
+    inp = I.make("tiny")
+    wl, T = inp.wl, inp.wl.temps[0]
+    w, g, a, b = bench.local_problem(inp.w, inp.g, rank, world, replicate)
+    soft_out = {}
+
+    def soft_fn(w_, c_):
+        soft_out["soft"] = oracle.soft(w_, c_, wl.L, wl.k, wl.V, T, nthreads=1)["soft"]
+
+    def vjp_fn(w_, c_, g_):
+        r = oracle.vjp(w_, c_, wl.L, wl.k, wl.V, T, g_, nthreads=1)
+        return torch.from_numpy(r["grad_w"]), torch.from_numpy(r["grad_c"]).clone()
+
+    first, second = bench.path_halves(soft_fn, vjp_fn, w, inp.c, g)
+    first()
+    gw, gc = second()
+    np.save(os.path.join(out_dir, f"b_soft{rank}.npy"), soft_out["soft"])
+    np.save(os.path.join(out_dir, f"b_gw{rank}.npy"), gw.numpy())
+    np.save(os.path.join(out_dir, f"b_gc{rank}.npy"), gc.numpy())
+    np.save(os.path.join(out_dir, f"b_rows{rank}.npy"), np.array([a, b]))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("replicate", [False, True])
+def test_bench_step_on_two_gloo_ranks(tmp_path, replicate):
+    """The bench's N > 1 step on CPU: sharded, the ranks' slices tile the
+    workload and the summed codebook gradient is the single-process one;
+    replicated, every rank holds the whole workload and the sum is twice it."""
+    import oracle
+    port = _free_port()
+    mp.start_processes(_bench_worker, args=(2, port, str(tmp_path), replicate), nprocs=2, join=True,
+                       start_method="spawn")
+    inp = I.make("tiny")
+    wl, T = inp.wl, inp.wl.temps[0]
+    ref_s = oracle.soft(inp.w, inp.c, wl.L, wl.k, wl.V, T, nthreads=1)["soft"]
+    ref = oracle.vjp(inp.w, inp.c, wl.L, wl.k, wl.V, T, inp.g, nthreads=1)
+    rows = [np.load(tmp_path / f"b_rows{r}.npy") for r in range(2)]
+    if replicate:
+        assert all(list(r) == [0, wl.n_seq] for r in rows)
+        soft = np.load(tmp_path / "b_soft0.npy")
+        gw = np.load(tmp_path / "b_gw0.npy")
+        gc_expect = 2 * ref["grad_c"]
+    else:
+        assert rows[0][0] == 0 and rows[0][1] == rows[1][0] and rows[1][1] == wl.n_seq
+        soft = np.concatenate([np.load(tmp_path / f"b_soft{r}.npy") for r in range(2)])
+        gw = np.concatenate([np.load(tmp_path / f"b_gw{r}.npy") for r in range(2)])
+        gc_expect = ref["grad_c"]
+    np.testing.assert_allclose(soft, ref_s, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(gw, ref["grad_w"], rtol=1e-12, atol=1e-12)
+    for r in range(2):
+        np.testing.assert_allclose(np.load(tmp_path / f"b_gc{r}.npy"), gc_expect, rtol=1e-12, atol=1e-12)
+
+
 def test_shard_rows_partition():
     for n in (0, 1, 7, 16, 16384):
         for world in (1, 2, 3, 8):

@@ -103,16 +103,31 @@ def test_empty_sequence_count_is_noop_and_zeroes_codebook_gradient():
     assert soft.numel() == 0 and float(gc.abs().max()) == 0.0
 
 
-def test_nan_sequence_is_isolated():
-    w, c, g = I.random_case(8, 2, 1, 5, 32, seed=77)
+@pytest.mark.parametrize("L,k,V", [(8, 2, 1), (16, 2, 1), (16, 2, 2)])
+def test_nan_sequence_is_isolated_and_flagged(L, k, V):
+    """A NaN weight makes its sequence's outputs NaN, leaves the others exact,
+    and the per-step posterior-mass check records BCJR_ERR_NUMERIC, which the
+    next read clears (generic, L=16 V=1 and V=2 kernels; soft and VJP)."""
+    w, c, g = I.random_case(L, k, V, 5, 32 * V, seed=77)
     w[2, 5] = float("nan")
-    soft, logZ = lib.soft_codeword(w.to(DEV), c.to(DEV), 8, 2, 1, 0.3)
-    soft, logZ = soft.cpu().numpy(), logZ.cpu().numpy()
-    assert np.isnan(logZ[2]) and np.isnan(soft[2]).any()
+    wd, cd, gd = w.to(DEV), c.to(DEV), g.to(DEV)
+    assert lib.get_device_error() == 0
+    soft, logZ = lib.soft_codeword(wd, cd, L, k, V, 0.3)
+    assert lib.get_device_error() == lib.BCJR_ERR_NUMERIC
+    assert lib.get_device_error() == 0
+    gw, _ = lib.vjp(wd, cd, L, k, V, 0.3, gd)
+    assert lib.get_device_error() == lib.BCJR_ERR_NUMERIC
+    soft, logZ, gw = soft.cpu().numpy(), logZ.cpu().numpy(), gw.cpu().numpy()
+    assert np.isnan(logZ[2]) and np.isnan(soft[2]).any() and np.isnan(gw[2]).any()
     ok = [0, 1, 3, 4]
-    ref = oracle.soft(w[ok], c, 8, 2, 1, 0.3)
-    assert_logZ(logZ[ok], ref["logZ"], 8, 2, 32)
+    ref = oracle.soft(w[ok], c, L, k, V, 0.3)
+    assert_logZ(logZ[ok], ref["logZ"], L, k * V, 32)
     assert_soft(soft[ok], ref["soft"], c)
+    rv = oracle.vjp(w[ok], c, L, k, V, 0.3, g[ok])
+    assert_grad(gw[ok], rv["grad_w"], "grad_w")
+    # a clean call afterwards leaves the flag clear
+    lib.soft_codeword(wd[ok[0]:ok[0] + 1].contiguous(), cd, L, k, V, 0.3)
+    assert lib.get_device_error() == 0
 
 
 def test_runs_are_bit_identical():

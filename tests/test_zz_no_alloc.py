@@ -37,7 +37,9 @@ def _call(fn, w, c, L, k, V, T, soft, logZ):
 
 
 @pytest.mark.parametrize("L,k,V,n_seq,n,T", [(8, 2, 1, 16, 64, 0.5), (12, 2, 1, 300, 256, 0.1),
-                                             (16, 2, 1, 20, 64, 0.05), (12, 2, 2, 9, 40, 0.05)])
+                                             (16, 2, 1, 20, 64, 0.05), (12, 2, 2, 9, 40, 0.05),
+                                             # 2^15 groups: the per-sequence state lives in the array too
+                                             (16, 1, 1, 8, 64, 0.1)])
 def test_noalloc_matches_allocating_entry_point(L, k, V, n_seq, n, T):
     fn = _noalloc()
     w, c, _ = I.random_case(L, k, V, n_seq, n * V, seed=4242 + L + V)
