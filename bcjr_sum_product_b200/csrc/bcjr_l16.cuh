@@ -30,15 +30,6 @@
 #pragma once
 #include "bcjr_kernels.cuh"
 
-// Prefetch distances of the VJP backward: codewords two units (8 states)
-// ahead, history vectors one block ahead.
-#ifndef BCJR_VJP_CB_AHEAD
-#define BCJR_VJP_CB_AHEAD 2
-#endif
-#ifndef BCJR_VJP_HOUT_AHEAD
-#define BCJR_VJP_HOUT_AHEAD 1
-#endif
-
 namespace bcjr {
 namespace l16 {
 
@@ -722,12 +713,9 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
     // that rounding carried along the recursions cancels in G.  Stored Bc_t is
     // relative to rB, the posterior mean of the previous step's stored values.
     float Kt = Hbar, rB = 0.f;
-    float cbn[8];
+    float cbn[8], cbm[8];
     ld_cb8(cs_tm, tid, 0, cbn);
-#if BCJR_VJP_CB_AHEAD == 2
-    float cbm[8];
     ld_cb8(cs_tm, tid, 1, cbm);
-#endif
     // block kk of step tt: A of step tt-1 in block-major order (free start: 0 for tt = 0)
     auto hist_a_at = [&](int tt, int kk) -> float4 {
       return (tt >= 1) ? reinterpret_cast<const float4*>(hist_a + (size_t)(tt - 1) * J)[tid + NT * kk]
@@ -741,9 +729,7 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
                        : make_float4(0.f, 0.f, 0.f, 0.f);
     };
     float4 hin_n = hist_l_at(n - 1, 0), han = hist_a_at(n - 1, 0);
-#if BCJR_VJP_HOUT_AHEAD
     float4 hout_n = POST ? hist_out(hist_l, n - 1, tid) : make_float4(0.f, 0.f, 0.f, 0.f);
-#endif
     float lsp = 0.f;     // log2 of the previous step's posterior mass (POST)
     float Rrn = 0.f;     // log domain: min of the previous step's stored values
     double Cr = 0.0;     // log domain: log2 beta_t = -stored + Cr_t
@@ -790,24 +776,15 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
           }
         }
         if (!last && k + 1 < KB) bvn = reinterpret_cast<const float4*>(bcur)[mid + NT];
-#if BCJR_VJP_HOUT_AHEAD
         const float4 hi4 = hin_n, ha4 = han, ho4 = hout_n;
-#else
-        const float4 hi4 = hin_n, ha4 = han;
-        const float4 ho4 = POST ? hist_out(hist_l, t, mid) : make_float4(0.f, 0.f, 0.f, 0.f);
-#endif
         if (k + 1 < KB) {
           hin_n = hist_l_at(t, k + 1);
           han = hist_a_at(t, k + 1);
-#if BCJR_VJP_HOUT_AHEAD
           if constexpr (POST) hout_n = hist_out(hist_l, t, mid + NT);
-#endif
         } else if (t >= 1) {
           hin_n = hist_l_at(t - 1, 0);
           han = hist_a_at(t - 1, 0);
-#if BCJR_VJP_HOUT_AHEAD
           if constexpr (POST) hout_n = hist_out(hist_l, t - 1, tid);
-#endif
         }
         float lnr[4];   // POST: n_t(j) + Rn_t - log2 mass
         if constexpr (POST) {
@@ -817,7 +794,6 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
 #pragma unroll
         for (int g = 0; g < 2; ++g) {          // groups h = 2g, 2g+1 side by side
           float cb[8];
-#if BCJR_VJP_CB_AHEAD == 2
 #pragma unroll
           for (int i = 0; i < 8; ++i) { cb[i] = cbn[i]; cbn[i] = cbm[i]; }
           {
@@ -825,15 +801,6 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
             const int nk = (k + 1 < KB) ? k + 1 : 0;
             ld_cb8(cs_tm, tid + NT * nk, g, cbm);
           }
-#else
-#pragma unroll
-          for (int i = 0; i < 8; ++i) cb[i] = cbn[i];
-          {
-            // codewords one unit after (k, g)
-            const int nk = g ? ((k + 1 < KB) ? k + 1 : 0) : k;
-            ld_cb8(cs_tm, tid + NT * nk, g ^ 1, cbn);
-          }
-#endif
           const float hs0 = g ? hi4.z : hi4.x, hs1 = g ? hi4.w : hi4.y;
           const float ha0 = g ? ha4.z : ha4.x, ha1 = g ? ha4.w : ha4.y;
           float gcb[8];
@@ -896,8 +863,8 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
             // underflows gets rho = 0 (+inf) and Bc = 0, moving no posterior by more than that mass
             nout[2 * g] = (kh.x - Rrn) - lg2f(ssum.x);
             nout[2 * g + 1] = (kh.y - Rrn) - lg2f(ssum.y);
-            bout[2 * g] = (ssum.x > 0.f) ? __fdividef(num.x, ssum.x) : 0.f;
-            bout[2 * g + 1] = (ssum.y > 0.f) ? __fdividef(num.y, ssum.y) : 0.f;
+            bout[2 * g] = __fdividef(num.x, fmaxf(ssum.x, FLT_MIN));   // num = 0 when sum p = 0
+            bout[2 * g + 1] = __fdividef(num.y, fmaxf(ssum.y, FLT_MIN));
             // posterior of the two step t-1 groups, P(i) = sum_lo p
             const float2 pg = ssum, bo = f2(bout[2 * g], bout[2 * g + 1]);
             accK = __ffma2_rn(pg, __fadd2_rn(f2(ha0, ha1), bo), accK);
