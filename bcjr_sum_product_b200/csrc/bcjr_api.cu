@@ -152,21 +152,40 @@ int grid_for(K kernel, int threads, size_t smem, int64_t n_seq, int* grid) {
   return BCJR_OK;
 }
 
-// Fewer resident CTAs when their per-CTA scratch (histories grow with the
-// sequence length) would exceed half of the free device memory or 24 GiB.
-void cap_grid_by_memory(int* grid, size_t per_cta_bytes) {
+// Scratch budget of one call: half of the free device memory, at most 24 GiB.
+size_t scratch_budget() {
   size_t free_b = 0, total_b = 0;
   if (cudaMemGetInfo(&free_b, &total_b) != cudaSuccess) {
     cudaGetLastError();
-    return;
+    return (size_t)1 << 30;
   }
-  size_t budget = free_b / 2;
   const size_t cap = (size_t)24 << 30;
-  if (budget > cap) budget = cap;
+  return free_b / 2 < cap ? free_b / 2 : cap;
+}
+
+// Fewer resident CTAs when their per-CTA scratch (histories grow with the
+// sequence length) would exceed the scratch budget.
+void cap_grid_by_memory(int* grid, size_t per_cta_bytes) {
   if (per_cta_bytes == 0) return;
-  size_t g = budget / per_cta_bytes;
+  size_t g = scratch_budget() / per_cta_bytes;
   if (g < 1) g = 1;
   if ((size_t)*grid > g) *grid = (int)g;
+}
+
+// Segment length of the checkpointed L = 16 histories: 0 (full histories)
+// while every resident CTA's full history fits the scratch budget, else
+// ceil(sqrt(n)).  BCJR_L16_CKPT=0 keeps full histories (fewer resident CTAs
+// instead); BCJR_L16_CKPT=K > 0 forces segments of K steps.
+int l16_checkpoint_len(int n, int grid, size_t full_bytes_per_cta) {
+  const char* e = std::getenv("BCJR_L16_CKPT");
+  if (e && e[0] != '\0') {
+    const long v = std::strtol(e, nullptr, 10);
+    if (v <= 0) return 0;
+    return (int)(v < n ? v : n);
+  }
+  if ((double)grid * (double)full_bytes_per_cta <= (double)scratch_budget()) return 0;
+  int K = (int)std::ceil(std::sqrt((double)n));
+  return K < 1 ? 1 : K;
 }
 
 // ----------------------------------------------------------------- sweep
@@ -204,6 +223,12 @@ struct SweepArgs {
 bool l16_vjp_cluster() {
   const char* e = std::getenv("BCJR_L16_VJP");
   return e && std::strcmp(e, "cluster") == 0;
+}
+// BCJR_L16_EX2=fma computes one of the three exponentials of each soft-pass
+// forward group on the FMA pipe (posterior-space soft kernel only).
+bool l16_fma_ex2() {
+  const char* e = std::getenv("BCJR_L16_EX2");
+  return e && std::strcmp(e, "fma") == 0;
 }
 bool l16_posterior_backward(bool vjp) {
   const char* e = std::getenv("BCJR_L16_BWD");
@@ -289,11 +314,21 @@ int run_l16(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
     if (rc != BCJR_ERR_UNSUPPORTED) return rc;
   }
   const bool post = l16_posterior_backward(VJP);
-  void (*kern)(K::Params) = post ? K::vjp_kernel<true> : K::vjp_kernel<false>;
-  if (!VJP) {
-    if (post) kern = a.out_argmax ? K::soft_kernel<true, true> : K::soft_kernel<false, true>;
-    else kern = a.out_argmax ? K::soft_kernel<true, false> : K::soft_kernel<false, false>;
-  }
+  const bool fma = post && l16_fma_ex2();
+  const bool am = a.out_argmax != nullptr;
+  auto pick = [&](bool ckpt) -> void (*)(K::Params) {
+#define BCJR_SOFT(AM, PO, FM) \
+  (ckpt ? K::soft_kernel<AM, PO, FM, true> : K::soft_kernel<AM, PO, FM, false>)
+    if (VJP) {
+      if (post) return ckpt ? K::vjp_kernel<true, true> : K::vjp_kernel<true, false>;
+      return ckpt ? K::vjp_kernel<false, true> : K::vjp_kernel<false, false>;
+    }
+    if (fma) return am ? BCJR_SOFT(true, true, true) : BCJR_SOFT(false, true, true);
+    if (post) return am ? BCJR_SOFT(true, true, false) : BCJR_SOFT(false, true, false);
+    return am ? BCJR_SOFT(true, false, false) : BCJR_SOFT(false, false, false);
+#undef BCJR_SOFT
+  };
+  void (*kern)(K::Params) = pick(false);
   // state ping-pong, per-warp partials, TMEM slot, per-step weights (and gradients)
   const size_t smem = sizeof(float) * ((size_t)2 * K::J + (VJP ? 2 * 32 * 8 : 64 + 2 * 32 * 2 + 64 + 64) + 4 +
                                        (VJP ? 2 : 1) * (size_t)sh.n);
@@ -301,13 +336,24 @@ int run_l16(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   int grid = 0;
   int rc = grid_for(kern, K::NT, smem, sh.n_seq, &grid);
   if (rc != BCJR_OK) return rc;
-  cap_grid_by_memory(&grid, sizeof(float) * (size_t)sh.n * K::J * (VJP ? 2 : 1) + (sizeof(double) + sizeof(float)) * sh.n +
+  // histories: full ([n][J] per CTA, twice for the VJP) or checkpointed (segments of ck steps)
+  const size_t full_cta = sizeof(float) * (size_t)sh.n * K::J * (VJP ? 2 : 1);
+  const int ck = l16_checkpoint_len(sh.n, grid, full_cta);
+  if (ck) {
+    kern = pick(true);
+    if ((rc = grid_for(kern, K::NT, smem, sh.n_seq, &grid)) != BCJR_OK) return rc;
+  }
+  const size_t nseg = ck ? (size_t)((sh.n + ck - 1) / ck) : 0;
+  const size_t hist_cta_floats =
+      ck ? (size_t)K::J * (VJP ? 2 * nseg + 2 * (size_t)ck + 6 : nseg + (size_t)ck + 1) : (size_t)sh.n * K::J;
+  cap_grid_by_memory(&grid, sizeof(float) * hist_cta_floats * (ck || !VJP ? 1 : 2) +
+                                (sizeof(double) + sizeof(float)) * sh.n +
                                 (VJP ? sizeof(float) * 2 * K::J + sizeof(double) * K::S : 0));
   K::Params P{};
   auto layout = [&](Arena& ar) {
     P.cs_tm = ar.take<float>(K::S);
-    P.hist_l = ar.take<float>((size_t)grid * sh.n * K::J);
-    P.hist_a = VJP ? ar.take<float>((size_t)grid * sh.n * K::J) : nullptr;
+    P.hist_l = ar.take<float>((size_t)grid * hist_cta_floats);
+    P.hist_a = (VJP && !ck) ? ar.take<float>((size_t)grid * hist_cta_floats) : nullptr;
     P.hist_c = ar.take<double>((size_t)grid * sh.n);
     P.hist_rn = ar.take<float>((size_t)grid * sh.n);
     P.bc_g = VJP ? ar.take<float>((size_t)grid * 2 * K::J) : nullptr;
@@ -322,7 +368,7 @@ int run_l16(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   layout(ar);
   P.w = a.w; P.gsoft = a.gsoft; P.gZ = a.gZ;
   P.out_soft = a.out_soft; P.out_logZ = a.out_logZ; P.out_argmax = a.out_argmax; P.grad_w = a.grad_w;
-  P.n_seq = sh.n_seq; P.len = sh.len; P.n = sh.n;
+  P.n_seq = sh.n_seq; P.len = sh.len; P.n = sh.n; P.ck = ck;
   P.sk = (float)std::sqrt(1.4426950408889634 / (double)a.T);
   P.two_over_T = (float)(2.0 / (double)a.T);
   K::make_block_codebook<<<K::S / 256, 256, 0, st>>>(a.c, P.sk, const_cast<float*>(P.cs_tm));

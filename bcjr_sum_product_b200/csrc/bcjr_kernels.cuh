@@ -419,6 +419,13 @@ __global__ void __launch_bounds__(kMaxThreads) bcjr_sweep_kernel(SweepParams P) 
       Cr += (double)Rr;
       Rr = -INFINITY;
       for (int w2 = 0; w2 < nwarps; ++w2) Rr = fmaxf(Rr, wmax[pb * 32 + w2]);
+      if constexpr (!VJP) {
+        // the same renormalisation as below: dividing out this step's posterior
+        // mass keeps the drift of later steps to their own rounding
+        float sp_ = 0.f;
+        for (int w2 = 0; w2 < nwarps; ++w2) sp_ += part[(pb * 32 + w2) * NPT + V];
+        Cr -= (double)lg2f(sp_);
+      }
       if constexpr (VJP) {
         float sk_ = 0.f, sb_ = 0.f, sp_ = 0.f;
         for (int w2 = 0; w2 < nwarps; ++w2) {

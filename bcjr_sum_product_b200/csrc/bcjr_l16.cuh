@@ -48,10 +48,11 @@ struct Params {
   int32_t* out_argmax;   // [n_seq][n] or null
   float* grad_w;         // [n_seq][len] (VJP)
   double* gc_part;       // [grid][65536] block-major (VJP)
-  float* hist_l;         // [grid][n][J]
+  float* hist_l;         // [grid][n][J], or the checkpoint layout when ck > 0
   float* hist_a;         // [grid][n][J] (VJP)
   double* hist_c;        // [grid][n]  fp64 offsets of the forward steps
   float* hist_rn;        // [grid][n]  re-centring value of each forward step
+  int ck;                // checkpoint segment length K, 0 = full histories
   float* bc_g;           // [grid][2][J] (VJP backward ping-pong)
   int64_t n_seq, len;
   int n;
@@ -124,14 +125,6 @@ __host__ __device__ constexpr int bidx(int h, int lo) { return 8 * (h >> 1) + 2 
 // memory, nothing to wait for.
 __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-// The backward of step t reads the history of step t - 1; at its start lanes
-// 0..7 of one warp ask for step t - 2's (64 KB, eight 8 KB blocks) so that it is
-// in L2, not HBM, when the per-thread loads of the next step are issued.
-__device__ __forceinline__ void prefetch_history(const float* hist, int t, int lane) {
-  constexpr uint32_t kChunk = J * sizeof(float) / 8;
-  if (t >= 2 && lane < 8)
-    prefetch_l2_bulk(reinterpret_cast<const char*>(hist + (size_t)(t - 2) * J) + lane * kChunk, kChunk);
 }
 
 __device__ __forceinline__ void ld_cb(const float* __restrict__ cs_tm, int mid, float (&c)[16]) {
@@ -212,31 +205,94 @@ __device__ __forceinline__ float bfly16_sum(float v) {
   return v;
 }
 
+// 2^x on the FMA pipe instead of the MUFU unit, for x <= 127 (the split-ex2
+// variant of the soft kernel).  Cody and Waite's range reduction x = n + f with
+// n = round(x), f in [-1/2, 1/2] (adding and subtracting 1.5 * 2^23 rounds x to
+// an integer held in the low mantissa bits), then 2^f by a degree-5 polynomial
+// fitted for relative error (ex2_poly.py: 2.0e-7 in fp32, the accuracy of
+// ex2.approx), scaled by 2^n through the exponent field.  x is clamped to
+// -126, so results that ex2.approx.ftz flushes to 0 come out below 2^-126.
+__device__ __forceinline__ float ex2_fma(float x) {
+  constexpr float kRound = 12582912.f;   // 1.5 * 2^23
+  x = fminf(fmaxf(x, -126.f), 127.f);
+  const float t = __fadd_rn(x, kRound);
+  const float f = __fsub_rn(x, __fsub_rn(t, kRound));
+  float p = fmaf(0.0013266970636323094f, f, 0.009675459936261177f);
+  p = fmaf(p, f, 0.05550742521882057f);
+  p = fmaf(p, f, 0.24022121727466583f);
+  p = fmaf(p, f, 0.6931469440460205f);
+  p = fmaf(p, f, 1.0000001192092896f);
+  const uint32_t n = (uint32_t)(__float_as_int(t) - 0x4B400000);
+  return __uint_as_float(__float_as_uint(p) + (n << 23));
+}
+
 // One forward group of the soft pass: x_h = d_h^2 + n_h for the four members
 // (h = 0..3 in two lane pairs); returns the negated log2 of sum_h 2^(-x_h)
 // re-centred by Rn.  The smallest x contributes 2^0 = 1 exactly, so only the
-// three others need an ex2: a min/max network picks them.
+// three others need an ex2: a min/max network picks them.  With FMA_EX2 one
+// of the three runs on the FMA pipe.
+template <bool FMA_EX2 = false>
 __device__ __forceinline__ float soft_group(float2 x01, float2 x23, float Rn) {
   const float l01 = fminf(x01.x, x01.y), h01 = fmaxf(x01.x, x01.y);
   const float l23 = fminf(x23.x, x23.y), h23 = fmaxf(x23.x, x23.y);
   const float m = fminf(l01, l23), M = fmaxf(l01, l23);
   const float2 a = __ffma2_rn(f2(h01, h23), f2s(-1.f), f2s(m));
-  const float s = (1.f + ex2f(m - M)) + (ex2f(a.x) + ex2f(a.y));
+  const float e1 = FMA_EX2 ? ex2_fma(m - M) : ex2f(m - M);
+  const float s = (1.f + e1) + (ex2f(a.x) + ex2f(a.y));
   return (m - Rn) - lg2f(s);
 }
 
+// Forward values kept for the backward sweep, per CTA.  For sequences whose
+// full history fits the scratch budget, every step's vector ([n][J]).
+// Otherwise (long sequences) checkpoints: the forward keeps the vector of
+// every K-th step and all vectors of the last segment; the backward, before it
+// enters each earlier segment, recomputes that segment's forward from its
+// checkpoint into the segment buffer (about 2 sqrt(n) vectors instead of n,
+// for one more forward sweep over all but the last segment).  The recompute
+// repeats the stored per-step re-centring values, so its vectors have the same
+// bits as the first forward's.
+template <bool CKPT>
+struct History {
+  float* full;   // [n][J] (full histories)
+  float* ckpt;   // [S][J]: vector s = the forward values of step s K - 1 (s >= 1)
+  float* seg;    // [K][J]: the forward values of steps s0 .. s0 + K - 1
+  int K, s0;     // segment length, first step of the segment in seg
+  // vector of step tt; with checkpoints tt >= s0 - 1 (below that: the checkpoint
+  // of the segment containing tt + 1, an in-bounds vector of another step)
+  __device__ __forceinline__ const float* at(int tt) const {
+    if constexpr (!CKPT) return full + (size_t)tt * J;
+    return (tt >= s0) ? seg + (size_t)(tt - s0) * J : ckpt + (size_t)((tt + 1) / K) * J;
+  }
+  __device__ __forceinline__ bool resident(int tt) const { return !CKPT || tt >= s0; }
+};
+
 // n_{tt-1}((h << 12) | mid) for h = 0..3 (zero for tt = 0: free start)
-__device__ __forceinline__ float4 hist_in(const float* hist, int tt, int mid) {
+template <bool CKPT>
+__device__ __forceinline__ float4 hist_in(const History<CKPT>& H, int tt, int mid) {
   if (tt < 1) return make_float4(0.f, 0.f, 0.f, 0.f);
-  const float* p = hist + (size_t)(tt - 1) * J + mid;
+  const float* p = H.at(tt - 1) + mid;
   return make_float4(p[0], p[1 << HB], p[2 << HB], p[3 << HB]);
 }
 // n_tt((mid << 2) | lo) for lo = 0..3
-__device__ __forceinline__ float4 hist_out(const float* hist, int tt, int mid) {
-  return reinterpret_cast<const float4*>(hist + (size_t)tt * J)[mid];
+template <bool CKPT>
+__device__ __forceinline__ float4 hist_out(const History<CKPT>& H, int tt, int mid) {
+  return reinterpret_cast<const float4*>(H.at(tt))[mid];
+}
+// The backward of step t reads step t - 1's vector; at its start lanes 0..7 of
+// one warp ask for step t - 2's (64 KB) so that it is in L2 for the next step.
+template <bool CKPT>
+__device__ __forceinline__ void prefetch_history(const History<CKPT>& H, int t, int lane) {
+  constexpr uint32_t kChunk = J * sizeof(float) / 8;
+  if (t >= 2 && lane < 8 && H.resident(t - 2))
+    prefetch_l2_bulk(reinterpret_cast<const char*>(H.at(t - 2)) + lane * kChunk, kChunk);
+}
+// Copies a J-vector with all threads of the CTA (the caller synchronises).
+__device__ __forceinline__ void copy_vec(float* dst, const float* src, int tid) {
+  for (int j = 4 * tid; j < J; j += 4 * NT)
+    *reinterpret_cast<float4*>(dst + j) = *reinterpret_cast<const float4*>(src + j);
 }
 
-template <bool ARGMAX, bool POST>
+template <bool ARGMAX, bool POST, bool FMA_EX2, bool CKPT>
 __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
   constexpr int NP = 2;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -253,7 +309,22 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
   uint32_t* tslot = reinterpret_cast<uint32_t*>(aidx + 64);  // [4]
   float* wsc = reinterpret_cast<float*>(tslot + 4);    // n
 
-  float* hist = P.hist_l + (size_t)blockIdx.x * n * J;   // [n][J] negated forward values, group order
+  // per-CTA history: full [n][J], or checkpoints [S][J], a segment [K][J] and a
+  // save slot [J] for the backward message while a segment is recomputed
+  History<CKPT> H{};
+  float* msave = nullptr;
+  int s_last = 0;
+  if constexpr (!CKPT) {
+    H.full = P.hist_l + (size_t)blockIdx.x * n * J;
+  } else {
+    const int K = P.ck, S = (n + K - 1) / K;
+    float* base = P.hist_l + (size_t)blockIdx.x * (S + K + 1) * J;
+    H.ckpt = base;
+    H.seg = base + (size_t)S * J;
+    msave = base + (size_t)(S + K) * J;
+    H.K = K;
+    s_last = ((n - 1) / K) * K;
+  }
   double* hist_c = P.hist_c + (size_t)blockIdx.x * n;
   float* hist_rn = P.hist_rn + (size_t)blockIdx.x * n;
   const float2 neg1 = f2s(-1.f);
@@ -271,44 +342,73 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
   }
   tmem_wait_st();
 
+  // One forward step: reads step t-1's vector from shared memory, writes step
+  // t's there and to up to two history slots; returns the thread's minimum of
+  // the stored values.
+  auto forward_step = [&](int t, float Rn, float* dst_a, float* dst_b) -> float {
+    const float* nprev = lb[(t + 1) & 1];
+    float* ncur = lb[t & 1];
+    const float2 nw2 = f2s(wsc[t]);
+    float tmin = INFINITY;
+#pragma unroll
+    for (int k = 0; k < KB; ++k) {
+      const int mid = tid + NT * k;
+      float cb[16];
+      tmem_ld16(tbase + 16 * k, cb);
+      float2 np01, np23;
+      if (t == 0) {
+        np01 = f2s(0.f); np23 = f2s(0.f);
+      } else {
+        np01 = f2(nprev[(0 << HB) | mid], nprev[(1 << HB) | mid]);
+        np23 = f2(nprev[(2 << HB) | mid], nprev[(3 << HB) | mid]);
+      }
+      float out[4];
+#pragma unroll
+      for (int lo = 0; lo < 4; ++lo) {
+        const float2 d01 = __fadd2_rn(f2(cb[bidx(0, lo)], cb[bidx(1, lo)]), nw2);
+        const float2 d23 = __fadd2_rn(f2(cb[bidx(2, lo)], cb[bidx(3, lo)]), nw2);
+        out[lo] = soft_group<FMA_EX2>(__ffma2_rn(d01, d01, np01), __ffma2_rn(d23, d23, np23), Rn);
+      }
+      tmin = fminf(tmin, fminf(fminf(out[0], out[1]), fminf(out[2], out[3])));
+      const float4 ov = make_float4(out[0], out[1], out[2], out[3]);
+      reinterpret_cast<float4*>(ncur)[mid] = ov;
+      if (dst_a) reinterpret_cast<float4*>(dst_a)[mid] = ov;
+      if (dst_b) reinterpret_cast<float4*>(dst_b)[mid] = ov;
+    }
+    return tmin;
+  };
+
+  // Before the backward of step t enters the segment below the one in H.seg:
+  // the message of step t is saved, that segment's forward recomputed from its
+  // checkpoint, and the message restored.
+  auto enter_segment = [&](int t) {
+    if constexpr (!CKPT) return;
+    copy_vec(msave, lb[t & 1], tid);
+    H.s0 -= H.K;
+    if (H.s0 > 0) copy_vec(lb[(H.s0 + 1) & 1], H.ckpt + (size_t)(H.s0 / H.K) * J, tid);
+    __syncthreads();
+    for (int tt = H.s0; tt < H.s0 + H.K; ++tt) {
+      forward_step(tt, hist_rn[tt], H.seg + (size_t)(tt - H.s0) * J, nullptr);
+      __syncthreads();
+    }
+    copy_vec(lb[t & 1], msave, tid);
+    __syncthreads();
+  };
+
   for (int64_t seq = blockIdx.x; seq < P.n_seq; seq += gridDim.x) {
     const float* wq = P.w + seq * P.len;
     for (int x = tid; x < n; x += NT) wsc[x] = -wq[x] * P.sk;   // -w'
+    H.s0 = CKPT ? s_last : 0;
     __syncthreads();
 
     // ------------------------------------------------------------ forward
     float Rn = 0.f;     // min of the previous step's stored (negated) values
     double C = 0.0;     // log2 sigma_t = -stored + C_t
     for (int t = 0; t < n; ++t) {
-      const float* nprev = lb[(t + 1) & 1];
-      float* ncur = lb[t & 1];
-      const float2 nw2 = f2s(wsc[t]);
       C -= (double)Rn;
-      float tmin = INFINITY;
-#pragma unroll
-      for (int k = 0; k < KB; ++k) {
-        const int mid = tid + NT * k;
-        float cb[16];
-        tmem_ld16(tbase + 16 * k, cb);
-        float2 np01, np23;
-        if (t == 0) {
-          np01 = f2s(0.f); np23 = f2s(0.f);
-        } else {
-          np01 = f2(nprev[(0 << HB) | mid], nprev[(1 << HB) | mid]);
-          np23 = f2(nprev[(2 << HB) | mid], nprev[(3 << HB) | mid]);
-        }
-        float out[4];
-#pragma unroll
-        for (int lo = 0; lo < 4; ++lo) {
-          const float2 d01 = __fadd2_rn(f2(cb[bidx(0, lo)], cb[bidx(1, lo)]), nw2);
-          const float2 d23 = __fadd2_rn(f2(cb[bidx(2, lo)], cb[bidx(3, lo)]), nw2);
-          out[lo] = soft_group(__ffma2_rn(d01, d01, np01), __ffma2_rn(d23, d23, np23), Rn);
-        }
-        tmin = fminf(tmin, fminf(fminf(out[0], out[1]), fminf(out[2], out[3])));
-        const float4 ov = make_float4(out[0], out[1], out[2], out[3]);
-        reinterpret_cast<float4*>(ncur)[mid] = ov;
-        reinterpret_cast<float4*>(hist + (size_t)t * J)[mid] = ov;
-      }
+      float* dst_a = !CKPT ? H.full + (size_t)t * J : (t >= s_last ? H.seg + (size_t)(t - s_last) * J : nullptr);
+      float* dst_b = (CKPT && (t + 1) % H.K == 0 && t + 1 < n) ? H.ckpt + (size_t)((t + 1) / H.K) * J : nullptr;
+      float tmin = forward_step(t, Rn, dst_a, dst_b);
       tmin = -warp_max(-tmin);
       if (lane == 0) wmin[(t & 1) * 32 + warp] = tmin;
       if (tid == 0) { hist_c[t] = C; hist_rn[t] = Rn; }
@@ -340,9 +440,14 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
     // ------------------------------------------------------------ backward
     if constexpr (POST) {
       // block kk of step tt: its inputs (scalars) and outputs (vector), one block ahead
-      float4 hin_n = hist_in(hist, n - 1, tid), hout_n = hist_out(hist, n - 1, tid);
+      float4 hin_n = hist_in(H, n - 1, tid), hout_n = hist_out(H, n - 1, tid);
       for (int t = n - 1; t >= 0; --t) {
-        if (warp == 0) prefetch_history(hist, t, lane);
+        if (CKPT && t == H.s0 - 1) {
+          enter_segment(t);
+          hin_n = hist_in(H, t, tid);
+          hout_n = hist_out(H, t, tid);
+        }
+        if (warp == 0) prefetch_history(H, t, lane);
         const float* pcur = lb[t & 1];
         float* pnext = lb[(t + 1) & 1];
         const float2 nw2 = f2s(wsc[t]);
@@ -357,11 +462,11 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
           tmem_ld16(tbase + 16 * k, cb);
           const float4 hi4 = hin_n, ho4 = hout_n;
           if (k + 1 < KB) {
-            hin_n = hist_in(hist, t, mid + NT);
-            hout_n = hist_out(hist, t, mid + NT);
+            hin_n = hist_in(H, t, mid + NT);
+            hout_n = hist_out(H, t, mid + NT);
           } else if (t >= 1) {
-            hin_n = hist_in(hist, t - 1, tid);
-            hout_n = hist_out(hist, t - 1, tid);
+            hin_n = hist_in(H, t - 1, tid);
+            hout_n = hist_out(H, t - 1, tid);
           }
           const float4 pv = reinterpret_cast<const float4*>(pcur)[mid];
           const float pl[4] = {pv.x, pv.y, pv.z, pv.w};
@@ -421,9 +526,13 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
     } else {
       float Rrn = 0.f;
       double Cr = 0.0;   // log2 beta_t = -stored + Cr_t
-      float4 hsn = hist_in(hist, n - 1, tid);
+      float4 hsn = hist_in(H, n - 1, tid);
       for (int t = n - 1; t >= 0; --t) {
-        if (warp == 0) prefetch_history(hist, t, lane);
+        if (CKPT && t == H.s0 - 1) {
+          enter_segment(t);
+          hsn = hist_in(H, t, tid);
+        }
+        if (warp == 0) prefetch_history(H, t, lane);
         const float* ncur = lb[t & 1];
         float* nnext = lb[(t + 1) & 1];
         const float2 nw2 = f2s(wsc[t]);
@@ -440,8 +549,8 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
           float cb[16];
           tmem_ld16(tbase + 16 * k, cb);
           const float hs[4] = {hsn.x, hsn.y, hsn.z, hsn.w};
-          if (k + 1 < KB) hsn = hist_in(hist, t, mid + NT);
-          else if (t >= 1) hsn = hist_in(hist, t - 1, tid);
+          if (k + 1 < KB) hsn = hist_in(H, t, mid + NT);
+          else if (t >= 1) hsn = hist_in(H, t - 1, tid);
           float nr[4];
           if (last) {
             nr[0] = nr[1] = nr[2] = nr[3] = 0.f;
@@ -545,7 +654,7 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
 // exchanges the negated log rho and Bc = W / P instead.  Both renormalise the
 // posterior mass of every step (its sum drifts from 1 by the rounding of the
 // two sweeps).
-template <bool POST>
+template <bool POST, bool CKPT>
 __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n = P.n;
@@ -561,8 +670,34 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
   float* wsc = reinterpret_cast<float*>(tslot + 4);    // n: -w'
   float* gsc = wsc + n;                                // n: g / sk
 
-  float* hist_l = P.hist_l + (size_t)blockIdx.x * n * J;
-  float* hist_a = P.hist_a + (size_t)blockIdx.x * n * J;
+  // Per-CTA histories (see History), full or checkpointed.  Full: the forward
+  // values [n][J] (group order for the posterior space backward, block-major
+  // inputs for the log-domain one) and A [n][J] (block-major inputs).
+  // Checkpoints: the forward values and A of every K-th step in group order
+  // [S][J] each, one segment of both histories [K][J] each, and save slots for
+  // the backward messages [2][J] and the codebook gradient [4][J] while a
+  // segment is recomputed.  Block-major input slots of step t live at index
+  // t - 1 (full) or t - s0 (segment).
+  History<CKPT> H{};
+  float *hl_full = nullptr, *ha_full = nullptr, *ck_a = nullptr, *sg_a = nullptr;
+  float *msave = nullptr, *gsave = nullptr;
+  int s_last = 0;
+  if constexpr (!CKPT) {
+    hl_full = P.hist_l + (size_t)blockIdx.x * n * J;
+    ha_full = P.hist_a + (size_t)blockIdx.x * n * J;
+    H.full = hl_full;
+  } else {
+    const int K = P.ck, S = (n + K - 1) / K;
+    float* base = P.hist_l + (size_t)blockIdx.x * (2 * S + 2 * K + 6) * J;
+    H.ckpt = base;
+    ck_a = base + (size_t)S * J;
+    H.seg = base + (size_t)2 * S * J;
+    sg_a = H.seg + (size_t)K * J;
+    msave = sg_a + (size_t)K * J;
+    gsave = msave + (size_t)2 * J;
+    H.K = K;
+    s_last = ((n - 1) / K) * K;
+  }
   double* hist_c = P.hist_c + (size_t)blockIdx.x * n;
   float* hist_rn = P.hist_rn + (size_t)blockIdx.x * n;
   float* bcg[2] = {P.bc_g + (size_t)blockIdx.x * 2 * J, P.bc_g + (size_t)blockIdx.x * 2 * J + J};
@@ -577,24 +712,12 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
   const uint32_t tbase = tslot[0] + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(128 * (warp >> 2));
   for (int x = tid; x < S; x += NT) gcp[x] = 0.0;
 
-  for (int64_t seq = blockIdx.x; seq < P.n_seq; seq += gridDim.x) {
-    const float* wq = P.w + seq * P.len;
-    const float* gq = P.gsoft + seq * P.len;
-    for (int x = tid; x < n; x += NT) { wsc[x] = -wq[x] * P.sk; gsc[x] = gq[x] / P.sk; }
-    // codewords into tensor memory for the forward
-#pragma unroll
-    for (int k = 0; k < KB; ++k) {
-      float c16[16];
-      ld_cb(cs_tm, tid + NT * k, c16);
-      tmem_st16(tbase + 16 * k, c16);
-    }
-    tmem_wait_st();
-    __syncthreads();
-
-    // ------------------------------------------------------------ forward
-    float Rn = 0.f;
-    double C = 0.0;
-    for (int t = 0; t < n; ++t) {
+  // One forward step: step t-1's forward values (shared memory) and A (global
+  // ping-pong) in, step t's out; history slots that are non-null receive step
+  // t-1's values in block-major order (in_l, in_a), step t's in group order
+  // (out_l) and the checkpoint copies (ck_lt, ck_at).  Returns the thread's
+  // minimum of the stored values.
+  auto forward_step = [&](int t, float Rn, float* in_l, float* in_a, float* out_l, float* ck_lt, float* ck_at) -> float {
       const float* nprev = lb[(t + 1) & 1];
       float* ncur = lb[t & 1];
       // A_t ping-pongs in global scratch (L2-resident); the history copy is block-major
@@ -607,7 +730,6 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
       // instead of growing with t; the histories keep the stored values and
       // the backward subtracts the same reference.
       const float2 nrA = f2s((t > 0) ? -aprev[0] : 0.f);
-      C -= (double)Rn;
       float tmin = INFINITY;
       float apn[4] = {0.f, 0.f, 0.f, 0.f};
       if (t > 0) {
@@ -633,9 +755,8 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
           np23 = f2(nprev[(2 << HB) | mid], nprev[(3 << HB) | mid]);
           // step t-1's values in block-major order [mid][h], as the backward reads them
           // (the posterior space backward takes the forward values in group order instead)
-          if constexpr (!POST)
-            reinterpret_cast<float4*>(hist_l + (size_t)(t - 1) * J)[mid] = make_float4(np01.x, np01.y, np23.x, np23.y);
-          reinterpret_cast<float4*>(hist_a + (size_t)(t - 1) * J)[mid] = make_float4(ap01.x, ap01.y, ap23.x, ap23.y);
+          if (in_l) reinterpret_cast<float4*>(in_l)[mid] = make_float4(np01.x, np01.y, np23.x, np23.y);
+          if (in_a) reinterpret_cast<float4*>(in_a)[mid] = make_float4(ap01.x, ap01.y, ap23.x, ap23.y);
         }
         float out[4], aout[4];
 #pragma unroll
@@ -655,10 +776,51 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
         }
         tmin = fminf(tmin, fminf(fminf(out[0], out[1]), fminf(out[2], out[3])));
         const float4 ov = make_float4(out[0], out[1], out[2], out[3]);
+        const float4 av = make_float4(aout[0], aout[1], aout[2], aout[3]);
         reinterpret_cast<float4*>(ncur)[mid] = ov;
-        if constexpr (POST) reinterpret_cast<float4*>(hist_l + (size_t)t * J)[mid] = ov;
-        reinterpret_cast<float4*>(acur)[mid] = make_float4(aout[0], aout[1], aout[2], aout[3]);
+        reinterpret_cast<float4*>(acur)[mid] = av;
+        if (out_l) reinterpret_cast<float4*>(out_l)[mid] = ov;
+        if (ck_lt) reinterpret_cast<float4*>(ck_lt)[mid] = ov;
+        if (ck_at) reinterpret_cast<float4*>(ck_at)[mid] = av;
       }
+    return tmin;
+  };
+
+  for (int64_t seq = blockIdx.x; seq < P.n_seq; seq += gridDim.x) {
+    const float* wq = P.w + seq * P.len;
+    const float* gq = P.gsoft + seq * P.len;
+    H.s0 = CKPT ? s_last : 0;
+    for (int x = tid; x < n; x += NT) { wsc[x] = -wq[x] * P.sk; gsc[x] = gq[x] / P.sk; }
+    // codewords into tensor memory for the forward
+#pragma unroll
+    for (int k = 0; k < KB; ++k) {
+      float c16[16];
+      ld_cb(cs_tm, tid + NT * k, c16);
+      tmem_st16(tbase + 16 * k, c16);
+    }
+    tmem_wait_st();
+    __syncthreads();
+
+    // ------------------------------------------------------------ forward
+    float Rn = 0.f;
+    double C = 0.0;
+    for (int t = 0; t < n; ++t) {
+      C -= (double)Rn;
+      float *in_l = nullptr, *in_a = nullptr, *out_l = nullptr, *ck_lt = nullptr, *ck_at = nullptr;
+      if constexpr (!CKPT) {
+        if (t >= 1) { in_l = POST ? nullptr : hl_full + (size_t)(t - 1) * J; in_a = ha_full + (size_t)(t - 1) * J; }
+        if (POST) out_l = hl_full + (size_t)t * J;
+      } else {
+        if (t >= s_last) {
+          if (t >= 1) { in_l = POST ? nullptr : H.seg + (size_t)(t - s_last) * J; in_a = sg_a + (size_t)(t - s_last) * J; }
+          if (POST) out_l = H.seg + (size_t)(t - s_last) * J;
+        }
+        if ((t + 1) % H.K == 0 && t + 1 < n) {
+          ck_lt = H.ckpt + (size_t)((t + 1) / H.K) * J;
+          ck_at = ck_a + (size_t)((t + 1) / H.K) * J;
+        }
+      }
+      float tmin = forward_step(t, Rn, in_l, in_a, out_l, ck_lt, ck_at);
       tmin = -warp_max(-tmin);
       if (lane == 0) rec[((t & 1) * 32 + warp) * 8 + 3] = tmin;
       if (tid == 0) { hist_c[t] = C; hist_rn[t] = Rn; }
@@ -716,25 +878,87 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
     float cbn[8], cbm[8];
     ld_cb8(cs_tm, tid, 0, cbn);
     ld_cb8(cs_tm, tid, 1, cbm);
+    // block-major input slot of step tt (tt >= 1), full or in the segment
+    auto in_slot = [&](const float* full, const float* seg, int tt) -> const float* {
+      if constexpr (!CKPT) return full + (size_t)(tt - 1) * J;
+      return seg + (size_t)(tt - H.s0) * J;
+    };
     // block kk of step tt: A of step tt-1 in block-major order (free start: 0 for tt = 0)
     auto hist_a_at = [&](int tt, int kk) -> float4 {
-      return (tt >= 1) ? reinterpret_cast<const float4*>(hist_a + (size_t)(tt - 1) * J)[tid + NT * kk]
+      return (tt >= 1) ? reinterpret_cast<const float4*>(in_slot(ha_full, sg_a, tt))[tid + NT * kk]
                        : make_float4(0.f, 0.f, 0.f, 0.f);
     };
     // forward values of step tt-1 for block kk: four scalars of the group-order
     // history (posterior space) or one vector of the block-major one (log domain)
     auto hist_l_at = [&](int tt, int kk) -> float4 {
-      if constexpr (POST) return hist_in(hist_l, tt, tid + NT * kk);
-      return (tt >= 1) ? reinterpret_cast<const float4*>(hist_l + (size_t)(tt - 1) * J)[tid + NT * kk]
+      if constexpr (POST) return hist_in(H, tt, tid + NT * kk);
+      return (tt >= 1) ? reinterpret_cast<const float4*>(in_slot(hl_full, H.seg, tt))[tid + NT * kk]
                        : make_float4(0.f, 0.f, 0.f, 0.f);
     };
+    // Before the backward of step t enters the segment below the one held: the
+    // messages of step t and the codebook gradient are saved, the codewords put
+    // back into tensor memory, that segment's forward recomputed from its
+    // checkpoint, and gradient and messages restored.
+    auto enter_segment = [&](int t) {
+      if constexpr (!CKPT) return;
+      copy_vec(msave, lb[t & 1], tid);
+      copy_vec(msave + J, bcg[t & 1], tid);
+#pragma unroll
+      for (int k = 0; k < KB; ++k) {
+        float v16[16];
+        tmem_ld16(tbase + 16 * k, v16);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) gsave[(size_t)(16 * k + i) * NT + tid] = v16[i];
+        ld_cb(cs_tm, tid + NT * k, v16);
+        tmem_st16(tbase + 16 * k, v16);
+      }
+      tmem_wait_st();
+      H.s0 -= H.K;
+      if (H.s0 > 0) {
+        copy_vec(lb[(H.s0 + 1) & 1], H.ckpt + (size_t)(H.s0 / H.K) * J, tid);
+        copy_vec(bcg[(H.s0 + 1) & 1], ck_a + (size_t)(H.s0 / H.K) * J, tid);
+      }
+      __syncthreads();
+      for (int tt = H.s0; tt < H.s0 + H.K; ++tt) {
+        float* sl = H.seg + (size_t)(tt - H.s0) * J;
+        float* sa = sg_a + (size_t)(tt - H.s0) * J;
+        forward_step(tt, hist_rn[tt], (!POST && tt >= 1) ? sl : nullptr, tt >= 1 ? sa : nullptr, POST ? sl : nullptr,
+                     nullptr, nullptr);
+        __syncthreads();
+      }
+#pragma unroll
+      for (int k = 0; k < KB; ++k) {
+        float v16[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v16[i] = gsave[(size_t)(16 * k + i) * NT + tid];
+        tmem_st16(tbase + 16 * k, v16);
+      }
+      tmem_wait_st();
+      copy_vec(lb[t & 1], msave, tid);
+      copy_vec(bcg[t & 1], msave + J, tid);
+      __syncthreads();
+    };
     float4 hin_n = hist_l_at(n - 1, 0), han = hist_a_at(n - 1, 0);
-    float4 hout_n = POST ? hist_out(hist_l, n - 1, tid) : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 hout_n = POST ? hist_out(H, n - 1, tid) : make_float4(0.f, 0.f, 0.f, 0.f);
     float lsp = 0.f;     // log2 of the previous step's posterior mass (POST)
     float Rrn = 0.f;     // log domain: min of the previous step's stored values
     double Cr = 0.0;     // log domain: log2 beta_t = -stored + Cr_t
     for (int t = n - 1; t >= 0; --t) {
-      if (warp == 0) prefetch_history(hist_l, t, lane);
+      if (CKPT && t == H.s0 - 1) {
+        enter_segment(t);
+        hin_n = hist_l_at(t, 0);
+        han = hist_a_at(t, 0);
+        if constexpr (POST) hout_n = hist_out(H, t, tid);
+      }
+      if (warp == 0) {
+        if constexpr (POST) {
+          prefetch_history(H, t, lane);
+        } else if (t >= 2 && lane < 8 && (!CKPT || t - 1 >= H.s0)) {
+          // the next step's block-major forward values (slot t - 2)
+          constexpr uint32_t kChunk = J * sizeof(float) / 8;
+          prefetch_l2_bulk(reinterpret_cast<const char*>(in_slot(hl_full, H.seg, t - 1)) + lane * kChunk, kChunk);
+        }
+      }
       const float* ncur = lb[t & 1];
       float* nnext = lb[(t + 1) & 1];
       const float* bcur = bcg[t & 1];
@@ -744,7 +968,7 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
       const float2 g2 = f2s(gsc[t]);
       const float2 gr2 = f2s(gsc[t] * P.sk);
       const bool last = (t == n - 1);
-      const float rA = (t >= 1) ? hist_a[(size_t)(t - 1) * J] : 0.f;   // the forward's reference
+      const float rA = (t >= 1) ? in_slot(ha_full, sg_a, t)[0] : 0.f;   // the forward's reference
       const float hbt = Kt + rA - rB - gzq;
       // POST: 2^(n_t + Rn_t - x) / (posterior mass); log domain: K = log2 of 1/Z and the offsets
       const float nrs = POST ? hist_rn[t] - lsp : 0.f;
@@ -780,11 +1004,11 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
         if (k + 1 < KB) {
           hin_n = hist_l_at(t, k + 1);
           han = hist_a_at(t, k + 1);
-          if constexpr (POST) hout_n = hist_out(hist_l, t, mid + NT);
+          if constexpr (POST) hout_n = hist_out(H, t, mid + NT);
         } else if (t >= 1) {
           hin_n = hist_l_at(t - 1, 0);
           han = hist_a_at(t - 1, 0);
-          if constexpr (POST) hout_n = hist_out(hist_l, t - 1, tid);
+          if constexpr (POST) hout_n = hist_out(H, t - 1, tid);
         }
         float lnr[4];   // POST: n_t(j) + Rn_t - log2 mass
         if constexpr (POST) {

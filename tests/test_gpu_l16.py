@@ -66,7 +66,7 @@ def _twice(fn):
 
 
 @pytest.mark.parametrize("variant", [{}, {"BCJR_L16_VJP": "cluster"}, {"BCJR_L16_BWD": "post"},
-                                     {"BCJR_L16_BWD": "log"}])
+                                     {"BCJR_L16_BWD": "log"}, {"BCJR_L16_EX2": "fma"}])
 def test_l16_v1_runs_are_bit_identical(monkeypatch, variant):
     """L=16, k=2, V=1: soft codeword, logZ, argmax and VJP of 200 sequences
     (more than one per CTA) give the same bits on every run."""
@@ -102,15 +102,17 @@ def test_l16_viterbi_runs_are_bit_identical(V):
 @pytest.mark.parametrize("T", [1.0, 0.05, 0.01])
 def test_l16_posterior_space_and_log_backward_agree_with_oracle(monkeypatch, T):
     """Both backward sweeps of the L=16 V=1 kernels (posterior space and log
-    domain, each selected for the soft codeword and the VJP) against the oracle on 12 sequences of 80 steps,
+    domain, each selected for the soft codeword and the VJP), and the soft
+    pass with one forward exponential per group on the FMA pipe, against the oracle on 12 sequences of 80 steps,
     with a logZ gradient: soft codeword, logZ, grad_w and grad_c."""
     w, c, g = I.random_case(16, 2, 1, 12, 80, seed=700 + int(100 * T))
     gZ = torch.randn(12, generator=torch.Generator().manual_seed(9))
     ref = oracle.soft(w, c, 16, 2, 1, T)
     rv = oracle.vjp(w, c, 16, 2, 1, T, g, gZ)
     wd, cd, gd, gzd = w.to(DEV), c.to(DEV), g.to(DEV), gZ.to(DEV)
-    for bwd in ("post", "log"):
+    for bwd, ex2 in (("post", "mufu"), ("log", "mufu"), ("post", "fma")):
         monkeypatch.setenv("BCJR_L16_BWD", bwd)
+        monkeypatch.setenv("BCJR_L16_EX2", ex2)
         soft, logZ = lib.soft_codeword(wd, cd, 16, 2, 1, T)
         gw, gc = lib.vjp(wd, cd, 16, 2, 1, T, gd, gzd)
         assert lib.get_device_error() == 0
@@ -131,3 +133,62 @@ def test_l16_block_argmax_against_oracle():
         mask = (ref["top2"][..., 0] - ref["top2"][..., 1]) > 1e-4
         assert mask.mean() > 0.5
         np.testing.assert_array_equal(am[mask], ref["argmax"][mask])
+
+
+@pytest.fixture(scope="module")
+def longest_low_t_case():
+    """Two sequences of len 8192 (the longest supported) at T = 0.01, the
+    second with a biased upstream gradient, and their oracle results (about
+    13 GB of host memory and two minutes per sequence)."""
+    w, c, g = I.random_case(16, 2, 1, 2, 8192, seed=781)
+    g[1] += 1.0
+    ref = oracle.soft(w, c, 16, 2, 1, 0.01, nthreads=2)
+    rv = oracle.vjp(w, c, 16, 2, 1, 0.01, g, nthreads=2)
+    return w, c, g, ref, rv
+
+
+@pytest.mark.parametrize("variant", [{}, {"BCJR_L16_BWD": "post"}, {"BCJR_L16_BWD": "log"},
+                                     {"BCJR_L16_EX2": "fma"}, {"BCJR_GENERIC_ONLY": "1"}])
+def test_l16_variants_longest_sequences_low_temperature(monkeypatch, variant, longest_low_t_case):
+    """len = 8192 at T = 0.01 with a biased upstream gradient, where the log
+    values reach hundreds of bits: every L=16 V=1 kernel variant (and the
+    generic kernels) against the oracle."""
+    w, c, g, ref, rv = longest_low_t_case
+    for key, val in variant.items():
+        monkeypatch.setenv(key, val)
+    wd, cd, gd = w.to(DEV), c.to(DEV), g.to(DEV)
+    soft, logZ = lib.soft_codeword(wd, cd, 16, 2, 1, 0.01)
+    gw, gc = lib.vjp(wd, cd, 16, 2, 1, 0.01, gd)
+    assert lib.get_device_error() == 0
+    assert_soft(soft.cpu().numpy(), ref["soft"], c)
+    assert_logZ(logZ.cpu().numpy(), ref["logZ"], 16, 2, 8192)
+    assert_grad(gw.cpu().numpy(), rv["grad_w"], "grad_w")
+    assert_grad(gc.cpu().numpy(), rv["grad_c"], "grad_c")
+
+
+@pytest.mark.parametrize("variant", [{}, {"BCJR_L16_BWD": "post"}, {"BCJR_L16_BWD": "log"}])
+@pytest.mark.parametrize("n,K", [(100, 7), (100, 10), (37, 1), (37, 37), (64, 8)])
+def test_l16_checkpointed_histories_are_bit_identical(monkeypatch, variant, n, K):
+    """Segments of K steps recomputed from checkpoints (ragged last segment,
+    K = 1, K = n) give the same bits as full histories: the recompute repeats
+    the forward with the stored re-centring values.  Soft codeword, logZ,
+    argmax and VJP; 160 sequences (more than one per CTA)."""
+    for key, val in variant.items():
+        monkeypatch.setenv(key, val)
+    w, c, g = I.random_case(16, 2, 1, 160, n, seed=1200 + n + K)
+    gZ = torch.randn(160, generator=torch.Generator().manual_seed(K))
+    wd, cd, gd, gzd = w.to(DEV), c.to(DEV), g.to(DEV), gZ.to(DEV)
+
+    def run():
+        out = list(lib.soft_codeword(wd, cd, 16, 2, 1, 0.05)) + [lib.posterior_argmax(wd, cd, 16, 2, 1, 0.05)]
+        out += list(lib.vjp(wd, cd, 16, 2, 1, 0.05, gd, gzd))
+        torch.cuda.synchronize()
+        assert lib.get_device_error() == 0
+        return out
+
+    monkeypatch.setenv("BCJR_L16_CKPT", "0")
+    full = run()
+    monkeypatch.setenv("BCJR_L16_CKPT", str(K))
+    ck = run()
+    for a, b in zip(full, ck):
+        assert torch.equal(a, b)
