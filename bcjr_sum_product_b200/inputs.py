@@ -16,6 +16,8 @@ Differentiable Relaxation of Trellis-Coded Weight Quantization", Abstract):
 * ``layer``   L=16, k=2, V=2, the seven matrices of one decoder layer
               (2x 2048^2, 2x 512x2048, 2x 8192x2048, 2048x8192), 256-weight rows
               (128 steps of 2 weights), T=0.05
+* ``long``    L=16, k=2, V=1, an 8192x2048 matrix cut into 8192-weight rows
+              (2048 sequences, the longest supported length), T=0.05
 
 Draw recipe: every tensor is drawn on the CPU with ``torch.Generator`` seeded
 as stated and ``torch.randn(..., dtype=float32)``.  The codebook uses seed 0
@@ -78,6 +80,7 @@ WORKLOADS = {
     "layer": Workload("layer", 16, 2, 2, 256,
                       ((2048, 2048), (2048, 2048), (512, 2048), (512, 2048),
                        (8192, 2048), (8192, 2048), (2048, 8192)), (0.05,), "soft+vjp"),
+    "long": Workload("long", 16, 2, 1, 8192, ((8192, 2048),), (0.05,), "soft+vjp"),
 }
 
 CODEBOOK_SEED = 0

@@ -11,13 +11,14 @@ seed 2).  Metric: state-updates/s = n_seq * n_steps * 2^L per step / time
 (weights/s reported alongside).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload qtip|mid|mlp|layer|tiny] [--temp T] [--qat | --viterbi]
+                    [--workload qtip|mid|mlp|layer|tiny|long] [--temp T] [--qat | --viterbi]
                     [--replicate]
 
 The default workload is the QTIP-scale one above.  ``--workload`` measures the
 other seeded workloads of the inputs module with the same timing rules (``mid``
 is forward only: soft codeword and logZ; ``mlp`` takes ``--temp`` from
-{1, 0.1, 0.01}).  ``--qat`` times one self-reconstruction QAT step per
+{1, 0.1, 0.01}; ``long`` cuts the mlp matrix into 8192-weight rows, where the
+L=16 kernels keep checkpointed histories).  ``--qat`` times one self-reconstruction QAT step per
 iteration instead (``bcjr_qat_step``: soft codeword, loss and its upstream
 gradient, VJP and the in-place SGD update of the weights, lr 1e-3).
 ``--viterbi`` times the T -> 0 hard decode (``viterbi_decode``, the
@@ -106,7 +107,9 @@ def measured_peaks():
 def kernel_variants() -> dict:
     """The library's kernel selectors as this process sees them (defaults spelled out)."""
     return {"l16_backward": os.environ.get("BCJR_L16_BWD", "post (soft), log (VJP)"),
-            "l16_vjp": os.environ.get("BCJR_L16_VJP", "one CTA per sequence")}
+            "l16_vjp": os.environ.get("BCJR_L16_VJP", "one CTA per sequence"),
+            "l16_ex2": os.environ.get("BCJR_L16_EX2", "mufu"),
+            "l16_histories": os.environ.get("BCJR_L16_CKPT", "full, or sqrt(n) checkpoints beyond the scratch budget")}
 
 
 class ClockSampler:
@@ -300,7 +303,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seqs", type=int, default=0,
                     help="profiling only: run on the first N sequences of the workload (not a bench number)")
-    ap.add_argument("--workload", default=None, choices=["qtip", "mid", "mlp", "layer", "tiny"])
+    ap.add_argument("--workload", default=None, choices=["qtip", "mid", "mlp", "layer", "tiny", "long"])
     ap.add_argument("--temp", type=float, default=None, help="temperature (one of the workload's)")
     grp = ap.add_mutually_exclusive_group()
     grp.add_argument("--qat", action="store_true", help="time bcjr_qat_step (self-reconstruction QAT step)")
