@@ -539,9 +539,54 @@ int run_viterbi_l16(const Shape& sh, const float* w, const float* c, int32_t* ou
   return BCJR_OK;
 }
 
+// L = 16, D = 4, V = 2: the Viterbi of bcjr_l16v2.cuh.
+int run_viterbi_l16v2(const Shape& sh, const float* w, const float* c, int32_t* out_states, float* out_cost,
+                      cudaStream_t st) {
+  namespace K = bcjr::l16v2;
+  const size_t smem = sizeof(float) * ((size_t)2 * K::J + 32 + 32 + 64 + 4 + 2 * (size_t)sh.n);
+  if (smem > kMaxDynSmem) return BCJR_ERR_UNSUPPORTED;
+  int grid = 0;
+  int rc = grid_for(K::viterbi_kernel, K::NT, smem, sh.n_seq, &grid);
+  if (rc != BCJR_OK) return rc;
+  // backpointer batch per CTA: up to 16 sequences, within about 2.5 GB in total
+  const size_t per_seq = (size_t)sh.n * K::NT;   // 32-bit words
+  int64_t tb = (int64_t)(2500000000ull / (sizeof(uint32_t) * (size_t)grid * per_seq));
+  if (tb > 16) tb = 16;
+  if (tb < 1) tb = 1;
+  K::VParams P{};
+  float4* cf = nullptr;
+  float4* cbk = nullptr;
+  float2* cf1 = nullptr;
+  float2* cb1 = nullptr;
+  auto layout = [&](Arena& ar) {
+    cf = ar.take<float4>(K::CB4);
+    cbk = ar.take<float4>(K::CB4);
+    cf1 = ar.take<float2>(K::CB4);
+    cb1 = ar.take<float2>(K::CB4);
+    P.bp = ar.take<uint32_t>((size_t)grid * tb * per_seq);
+  };
+  Arena sizing;
+  layout(sizing);
+  void* mem = nullptr;
+  if (int arc = scratch_alloc(&mem, sizing.off, st)) return arc;
+  Arena ar;
+  ar.base = static_cast<char*>(mem);
+  layout(ar);
+  P.w = w; P.cf = cf; P.cf1 = cf1; P.out_states = out_states; P.out_cost = out_cost;
+  P.n_seq = sh.n_seq; P.len = sh.len; P.n = sh.n; P.tb = (int)tb;
+  K::make_codebooks<<<K::CB4 / 256, 256, 0, st>>>(c, 1.0f, cf, cbk, cf1, cb1);   // raw codewords
+  K::viterbi_kernel<<<grid, K::NT, smem, st>>>(P);
+  cudaError_t le = cudaGetLastError();
+  cudaError_t fe = cudaFreeAsync(mem, st);
+  if (le != cudaSuccess || fe != cudaSuccess) return BCJR_ERR_CUDA;
+  return BCJR_OK;
+}
+
 int run_viterbi(const Shape& sh, const float* w, const float* c, int32_t* out_states, float* out_cost,
                 cudaStream_t st) {
   if (sh.L == 16 && sh.D == 2 && sh.V == 1 && !generic_only()) return run_viterbi_l16(sh, w, c, out_states, out_cost, st);
+  if (sh.L == 16 && sh.D == 4 && sh.V == 2 && !generic_only())
+    return run_viterbi_l16v2(sh, w, c, out_states, out_cost, st);
   ViterbiKernel kern = pick_viterbi(sh.V, sh.D);
   if (!kern) return BCJR_ERR_UNSUPPORTED;
   const int threads = threads_for(sh.J, sh.B);

@@ -564,8 +564,7 @@ __global__ void __launch_bounds__(kMaxThreads) viterbi_kernel(ViterbiParams P) {
         for (int b = 0; b < B; ++b) {
           const int s = j | (b << HI);
           float c[V];
-#pragma unroll
-          for (int v = 0; v < V; ++v) c[v] = __ldg(P.c + (size_t)s * V + v);
+          load_cw<V>(P.c, s, c);   // one vector load per codeword
           const float qv = qcost<V>(wt, c);
           const float dlt = (t == 0) ? qv : __fadd_rn(mprev[s >> D], qv);
           if (dlt < best) { best = dlt; bb = b; }

@@ -659,5 +659,157 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
   if (warp == 0) l16::tmem_dealloc512(tslot[0]);
 }
 
+// ------------------------------------------------------------ Viterbi
+// The T -> 0 decode in the same layout: per step and forward group
+// j = (mid << 4) | lo, mu_t(j) = min_h delta_t((h << 12) | j) with
+// delta_t(q) = fl(mu_{t-1}(q >> 4) + cost_t(q)) (delta_0 = cost_0) and
+// cost_t(q) = fl(fl(fl(w0 - c0)^2) + fl(fl(w1 - c1)^2)), the lowest h winning
+// ties.  All of a thread's 8 groups read the same 16 predecessor values
+// mu_{t-1}((h << 8) | mid), once per step.  Component 0 of the raw codewords
+// sits in tensor memory (the thread's 128 states = its 128 columns),
+// component 1 streams from the forward-order copy in L2.  The 4-bit
+// backpointers of a thread's 8 groups form one 32-bit word per step.  A CTA
+// decodes a batch of up to TB sequences, then traces them back in parallel
+// (one thread per sequence).  The arithmetic is the prescribed fp32 sequence
+// in scalar IEEE round-to-nearest operations that are never fused.
+struct VParams {
+  const float* w;        // [n_seq][len], len = 2 n
+  const float4* cf;      // forward-order raw codebook (make_codebooks with scale 1)
+  const float2* cf1;     // its component 1
+  int32_t* out_states;   // [n_seq][n]
+  float* out_cost;       // [n_seq] or null
+  uint32_t* bp;          // [grid][TB][n][NT]
+  int64_t n_seq, len;
+  int n, tb;
+};
+
+__global__ void __launch_bounds__(NT, 1) viterbi_kernel(VParams P) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int nwarps = NT / 32;
+  const int n = P.n, TB = P.tb;
+  const int mid = tid >> 1, e = tid & 1;
+  extern __shared__ __align__(16) float smem[];
+  float* mb[2] = {smem, smem + J};
+  float* redv = smem + 2 * J;                          // [32]
+  int* redq = reinterpret_cast<int*>(redv + 32);       // [32]
+  int* fin = redq + 32;                                // [TB <= 64] final state per sequence of the batch
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(fin + 64);  // [4]
+  float* wsm = reinterpret_cast<float*>(tslot + 4);    // 2 n: w
+  uint32_t* bp = P.bp + (size_t)blockIdx.x * TB * n * NT;
+
+  if (warp == 0) l16::tmem_alloc512(tslot);
+  l16::tmem_fence_before();
+  __syncthreads();
+  l16::tmem_fence_after();
+  const uint32_t tbase = tslot[0] + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(128 * (warp >> 2));
+  stage_c0(P.cf + tid, tbase);
+  const float2* __restrict__ c1p = P.cf1 + tid;
+
+  const int64_t stride = (int64_t)gridDim.x;
+  for (int64_t base = blockIdx.x; base < P.n_seq; base += stride * TB) {
+    int nb = 0;
+    for (int i = 0; i < TB; ++i, ++nb) {
+      const int64_t seq = base + i * stride;
+      if (seq >= P.n_seq) break;
+      const float* wq = P.w + seq * P.len;
+      for (int x = tid; x < 2 * n; x += NT) wsm[x] = wq[x];
+      __syncthreads();
+      uint32_t* bpi = bp + (size_t)i * n * NT;
+      float bestv = INFINITY;
+      int bestq = 0x7fffffff;
+      for (int t = 0; t < n; ++t) {
+        const float* mprev = mb[(t + 1) & 1];
+        float* mcur = mb[t & 1];
+        const float w0 = wsm[2 * t], w1 = wsm[2 * t + 1];
+        const bool last = (t == n - 1);
+        float mu[16];
+#pragma unroll
+        for (int h = 0; h < 16; ++h) mu[h] = (t > 0) ? mprev[(h << 8) | mid] : 0.f;
+        float2 c1n[8];
+#pragma unroll
+        for (int p = 0; p < 8; ++p) c1n[p] = __ldg(c1p + p * NT);
+        float mout[G];
+        uint32_t word = 0;
+#pragma unroll
+        for (int k = 0; k < G; ++k) {
+          float c0[16];
+          l16::tmem_ld16(tbase + 16 * k, c0);
+          float2 c1[8];
+#pragma unroll
+          for (int p = 0; p < 8; ++p) c1[p] = c1n[p];
+          if (k + 1 < G) {
+#pragma unroll
+            for (int p = 0; p < 8; ++p) c1n[p] = __ldg(c1p + ((k + 1) * 8 + p) * NT);
+          }
+          float b = INFINITY;
+          uint32_t bh = 0;
+#pragma unroll
+          for (int h = 0; h < 16; ++h) {
+            const float d0 = __fsub_rn(w0, c0[h]);
+            const float d1 = __fsub_rn(w1, (h & 1) ? c1[h >> 1].y : c1[h >> 1].x);
+            const float q = __fadd_rn(__fmul_rn(d0, d0), __fmul_rn(d1, d1));
+            const float dl = (t > 0) ? __fadd_rn(mu[h], q) : q;
+            if (dl < b) { b = dl; bh = (uint32_t)h; }
+            if (last) {
+              const int qs = (h << 12) | (mid << 4) | (8 * e + k);
+              if (dl < bestv || (dl == bestv && qs < bestq)) { bestv = dl; bestq = qs; }
+            }
+          }
+          mout[k] = b;
+          word |= bh << (4 * k);
+        }
+        reinterpret_cast<float4*>(mcur + (mid << 4) + 8 * e)[0] = make_float4(mout[0], mout[1], mout[2], mout[3]);
+        reinterpret_cast<float4*>(mcur + (mid << 4) + 8 * e)[1] = make_float4(mout[4], mout[5], mout[6], mout[7]);
+        if (!last) bpi[(size_t)t * NT + tid] = word;
+        __syncthreads();
+      }
+      // argmin of delta_{n-1} over all states, lowest state on ties
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float v2 = __shfl_xor_sync(0xffffffffu, bestv, o);
+        const int q2 = __shfl_xor_sync(0xffffffffu, bestq, o);
+        if (v2 < bestv || (v2 == bestv && q2 < bestq)) { bestv = v2; bestq = q2; }
+      }
+      if (lane == 0) { redv[warp] = bestv; redq[warp] = bestq; }
+      __syncthreads();
+      if (tid == 0) {
+        float bv = INFINITY;
+        int bq = 0x7fffffff;
+#pragma unroll
+        for (int w2 = 0; w2 < nwarps; ++w2)
+          if (redv[w2] < bv || (redv[w2] == bv && redq[w2] < bq)) { bv = redv[w2]; bq = redq[w2]; }
+        if (bq == 0x7fffffff) bq = 0;  // all-NaN sequence
+        fin[i] = bq;
+        if (P.out_cost) P.out_cost[seq] = bv;
+      }
+      __syncthreads();
+    }
+    // trace the batch back, one thread per sequence: the state at step t is
+    // the backpointer's h of group s_{t+1} >> 4 at step t, above that group
+    if (tid < nb) {
+      const int i = tid;
+      const int64_t seq = base + i * stride;
+      const uint32_t* bpi = bp + (size_t)i * n * NT;
+      int32_t* out = P.out_states + seq * n;
+      int st = fin[i];
+      for (int t = n - 1; t >= 0; --t) {
+        out[t] = st;
+        if (t > 0) {
+          const int jp = st >> 4;   // group (mid' << 4) | lo' of the predecessors at step t-1
+          const int tau = ((jp >> 4) << 1) | ((jp & 15) >> 3);
+          const int h = (bpi[(size_t)(t - 1) * NT + tau] >> (4 * (jp & 7))) & 15;
+          st = jp | (h << 12);
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  l16::tmem_fence_before();
+  __syncthreads();
+  l16::tmem_fence_after();
+  if (warp == 0) l16::tmem_dealloc512(tslot[0]);
+}
+
 }  // namespace l16v2
 }  // namespace bcjr

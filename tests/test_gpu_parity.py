@@ -251,6 +251,24 @@ def test_l16_viterbi_matches_generic_and_oracle(monkeypatch):
     np.testing.assert_array_equal(c_fast[:6].cpu().numpy(), ref["cost"])
 
 
+def test_l16v2_viterbi_matches_generic_and_oracle(monkeypatch):
+    """The L=16, V=2 Viterbi (16 branches, 4-bit backpointers, batched traceback)
+    against the generic kernel (bit-exact) on 40 sequences of 64 steps, with exact
+    ties from a coarse codebook, and against the oracle on 6 of them."""
+    w, c, _ = I.random_case(16, 2, 2, 40, 128, seed=516)
+    c[::5] = torch.round(c[::5] * 4) / 4
+    w[:5] = torch.round(w[:5] * 4) / 4
+    wd, cd = w.to(DEV), c.to(DEV)
+    s_fast, c_fast = lib.viterbi_decode(wd, cd, 16, 2, 2)
+    monkeypatch.setenv("BCJR_GENERIC_ONLY", "1")
+    s_gen, c_gen = lib.viterbi_decode(wd, cd, 16, 2, 2)
+    torch.cuda.synchronize()
+    assert torch.equal(s_fast, s_gen) and torch.equal(c_fast, c_gen)
+    ref = oracle.viterbi(w[:6], c, 16, 2, 2)
+    np.testing.assert_array_equal(s_fast[:6].cpu().numpy(), ref["states"])
+    np.testing.assert_array_equal(c_fast[:6].cpu().numpy(), ref["cost"])
+
+
 def test_longest_sequences(monkeypatch):
     """len = 8192 (the largest supported): L=12 against the oracle, and L=16
     (whose per-CTA histories are 0.5-1 GB, so fewer CTAs are resident) against
