@@ -508,18 +508,23 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
           if constexpr (ARGMAX) { apart[pb * 32 + warp] = bestp; aidx[pb * 32 + warp] = bestq; }
         }
         __syncthreads();
-        if (tid == 0) {
-          float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-          for (int w2 = 0; w2 < nwarps; ++w2) { s0 += part[(pb * 32 + w2) * NP]; s1 += part[(pb * 32 + w2) * NP + 1]; }
-          check_posterior_mass(s1);
-          if (P.out_soft) P.out_soft[seq * P.len + t] = s0 / (s1 * P.sk);
+        if (warp == 0) {   // the 16 partials combined by a butterfly: no serial tail before the next step
+          const float s0 = bfly16_sum(part[(pb * 32 + (lane & 15)) * NP]);
+          const float s1 = bfly16_sum(part[(pb * 32 + (lane & 15)) * NP + 1]);
+          if (lane == 0) {
+            check_posterior_mass(s1);
+            if (P.out_soft) P.out_soft[seq * P.len + t] = s0 / (s1 * P.sk);
+          }
           if constexpr (ARGMAX) {
-            float bp = -1.f;
-            int bq = 0x7fffffff;
+            float bp = apart[pb * 32 + (lane & 15)];
+            int bq = aidx[pb * 32 + (lane & 15)];
 #pragma unroll
-            for (int w2 = 0; w2 < nwarps; ++w2) arg_better(bp, bq, apart[pb * 32 + w2], aidx[pb * 32 + w2]);
-            if (P.out_argmax) P.out_argmax[seq * n + t] = bq;
+            for (int o = 8; o > 0; o >>= 1) {
+              const float p2 = __shfl_xor_sync(0xffffffffu, bp, o);
+              const int q2 = __shfl_xor_sync(0xffffffffu, bq, o);
+              arg_better(bp, bq, p2, q2);
+            }
+            if (lane == 0 && P.out_argmax) P.out_argmax[seq * n + t] = bq;
           }
         }
       }
@@ -605,18 +610,23 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
           if constexpr (ARGMAX) { apart[pb * 32 + warp] = bestp; aidx[pb * 32 + warp] = bestq; }
         }
         __syncthreads();
-        if (tid == 0) {
-          float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-          for (int w2 = 0; w2 < nwarps; ++w2) { s0 += part[(pb * 32 + w2) * NP]; s1 += part[(pb * 32 + w2) * NP + 1]; }
-          check_posterior_mass(s1);
-          if (P.out_soft) P.out_soft[seq * P.len + t] = s0 / (s1 * P.sk);
+        if (warp == 0) {   // the 16 partials combined by a butterfly: no serial tail before the next step
+          const float s0 = bfly16_sum(part[(pb * 32 + (lane & 15)) * NP]);
+          const float s1 = bfly16_sum(part[(pb * 32 + (lane & 15)) * NP + 1]);
+          if (lane == 0) {
+            check_posterior_mass(s1);
+            if (P.out_soft) P.out_soft[seq * P.len + t] = s0 / (s1 * P.sk);
+          }
           if constexpr (ARGMAX) {
-            float bp = -1.f;
-            int bq = 0x7fffffff;
+            float bp = apart[pb * 32 + (lane & 15)];
+            int bq = aidx[pb * 32 + (lane & 15)];
 #pragma unroll
-            for (int w2 = 0; w2 < nwarps; ++w2) arg_better(bp, bq, apart[pb * 32 + w2], aidx[pb * 32 + w2]);
-            if (P.out_argmax) P.out_argmax[seq * n + t] = bq;
+            for (int o = 8; o > 0; o >>= 1) {
+              const float p2 = __shfl_xor_sync(0xffffffffu, bp, o);
+              const int q2 = __shfl_xor_sync(0xffffffffu, bq, o);
+              arg_better(bp, bq, p2, q2);
+            }
+            if (lane == 0 && P.out_argmax) P.out_argmax[seq * n + t] = bq;
           }
         }
         Cr -= (double)Rrn;
