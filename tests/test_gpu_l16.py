@@ -99,13 +99,13 @@ def test_l16_viterbi_runs_are_bit_identical(V):
         assert torch.equal(x, y)
 
 
-@pytest.mark.parametrize("T", [1.0, 0.05, 0.01])
+@pytest.mark.parametrize("T", [1.0, 0.05, 0.01, 0.001])
 def test_l16_posterior_space_and_log_backward_agree_with_oracle(monkeypatch, T):
     """Both backward sweeps of the L=16 V=1 kernels (posterior space and log
     domain, each selected for the soft codeword and the VJP), and the soft
     pass with one forward exponential per group on the FMA pipe, against the oracle on 12 sequences of 80 steps,
     with a logZ gradient: soft codeword, logZ, grad_w and grad_c."""
-    w, c, g = I.random_case(16, 2, 1, 12, 80, seed=700 + int(100 * T))
+    w, c, g = I.random_case(16, 2, 1, 12, 80, seed=700 + int(1000 * T))
     gZ = torch.randn(12, generator=torch.Generator().manual_seed(9))
     ref = oracle.soft(w, c, 16, 2, 1, T)
     rv = oracle.vjp(w, c, 16, 2, 1, T, g, gZ)

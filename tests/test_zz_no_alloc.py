@@ -13,6 +13,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from bcjr_sum_product_b200 import inputs as I
 from bcjr_sum_product_b200 import lib
 from helpers import assert_logZ, assert_soft
@@ -39,7 +40,9 @@ def _call(fn, w, c, L, k, V, T, soft, logZ):
 @pytest.mark.parametrize("L,k,V,n_seq,n,T", [(8, 2, 1, 16, 64, 0.5), (12, 2, 1, 300, 256, 0.1),
                                              (16, 2, 1, 20, 64, 0.05), (12, 2, 2, 9, 40, 0.05),
                                              # 2^15 groups: the per-sequence state lives in the array too
-                                             (16, 1, 1, 8, 64, 0.1)])
+                                             (16, 1, 1, 8, 64, 0.1),
+                                             # 16 branches, where bcjr_soft_codeword runs a specialised kernel
+                                             (16, 2, 2, 9, 32, 0.05)])
 def test_noalloc_matches_allocating_entry_point(L, k, V, n_seq, n, T):
     fn = _noalloc()
     w, c, _ = I.random_case(L, k, V, n_seq, n * V, seed=4242 + L + V)
@@ -64,3 +67,18 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     soft = torch.empty_like(w)
     logZ = torch.empty(1, device="cuda")
     assert _call(fn, w, c, 16, 2, 1, 0.5, soft, logZ) == lib.BCJR_ERR_UNSUPPORTED
+
+
+def test_noalloc_against_the_oracle():
+    """The entry point's own results against the fp64 oracle (L=12 and L=16 V=2)."""
+    fn = _noalloc()
+    for L, k, V, n_seq, n, T in ((12, 2, 1, 20, 48, 0.1), (16, 2, 2, 3, 16, 0.05)):
+        w, c, _ = I.random_case(L, k, V, n_seq, n * V, seed=77 + L)
+        soft = torch.empty((n_seq, n * V), device="cuda")
+        logZ = torch.empty(n_seq, device="cuda")
+        assert _call(fn, w.cuda(), c.cuda(), L, k, V, T, soft, logZ) == lib.BCJR_OK
+        torch.cuda.synchronize()
+        assert lib.get_device_error() == 0
+        ref = oracle.soft(w, c, L, k, V, T)
+        assert_logZ(logZ.cpu().numpy(), ref["logZ"], L, k * V, n)
+        assert_soft(soft.cpu().numpy(), ref["soft"], c)
