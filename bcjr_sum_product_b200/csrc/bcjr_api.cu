@@ -217,12 +217,24 @@ struct SweepArgs {
 
 // Measured alternatives of the L = 16, k = 2, V = 1 kernels, selected per call.
 // BCJR_L16_VJP=cluster runs the VJP on clusters of two CTAs (bcjr_l16c.cuh)
-// instead of one CTA per sequence.  The backward sweeps run in posterior space
-// for the soft codeword and in log domain for the VJP (the faster of the two for
-// each); BCJR_L16_BWD=post or =log selects one of them for both.
+// instead of one CTA per sequence; BCJR_L16_VJP=l2 streams the VJP backward's
+// codewords from L2 instead of the shared-memory ring (the ring is the default
+// wherever it fits: full histories and shared memory).  The backward sweeps run
+// in posterior space for the soft codeword and in log domain for the VJP (the
+// faster of the two for each); BCJR_L16_BWD=post or =log selects one of them for
+// both.  BCJR_L16_RING_TEST_NOFILL=1 (tests only) never fills the ring, so that
+// its bounded waits run out and the call reports BCJR_ERR_TIMEOUT.
 bool l16_vjp_cluster() {
   const char* e = std::getenv("BCJR_L16_VJP");
   return e && std::strcmp(e, "cluster") == 0;
+}
+bool l16_vjp_ring() {
+  const char* e = std::getenv("BCJR_L16_VJP");
+  return !(e && std::strcmp(e, "l2") == 0);
+}
+bool l16_ring_test_nofill() {
+  const char* e = std::getenv("BCJR_L16_RING_TEST_NOFILL");
+  return e && std::strcmp(e, "1") == 0;
 }
 // BCJR_L16_EX2=fma computes one of the three exponentials of each soft-pass
 // forward group on the FMA pipe (posterior-space soft kernel only).
@@ -316,23 +328,30 @@ int run_l16(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   const bool post = l16_posterior_backward(VJP);
   const bool fma = post && l16_fma_ex2();
   const bool am = a.out_argmax != nullptr;
-  auto pick = [&](bool ckpt) -> void (*)(K::Params) {
+  auto pick = [&](bool ckpt, bool ring) -> void (*)(K::Params) {
 #define BCJR_SOFT(AM, PO, FM) \
   (ckpt ? K::soft_kernel<AM, PO, FM, true> : K::soft_kernel<AM, PO, FM, false>)
     if (VJP) {
-      if (post) return ckpt ? K::vjp_kernel<true, true> : K::vjp_kernel<true, false>;
-      return ckpt ? K::vjp_kernel<false, true> : K::vjp_kernel<false, false>;
+      if (ckpt) return post ? K::vjp_kernel<true, true, false> : K::vjp_kernel<false, true, false>;
+      if (post) return ring ? K::vjp_kernel<true, false, true> : K::vjp_kernel<true, false, false>;
+      return ring ? K::vjp_kernel<false, false, true> : K::vjp_kernel<false, false, false>;
     }
     if (fma) return am ? BCJR_SOFT(true, true, true) : BCJR_SOFT(false, true, true);
     if (post) return am ? BCJR_SOFT(true, true, false) : BCJR_SOFT(false, true, false);
     return am ? BCJR_SOFT(true, false, false) : BCJR_SOFT(false, false, false);
 #undef BCJR_SOFT
   };
-  void (*kern)(K::Params) = pick(false);
-  // state ping-pong, per-warp partials, TMEM slot, per-step weights (and gradients)
-  const size_t smem = sizeof(float) * ((size_t)2 * K::J + (VJP ? 2 * 32 * 8 : 64 + 2 * 32 * 2 + 64 + 64) + 4 +
-                                       (VJP ? 2 : 1) * (size_t)sh.n);
+  // state ping-pong, per-warp partials, TMEM slot, per-step weights (and gradients),
+  // and for the VJP with the codeword ring its stages and their control words
+  auto smem_for = [&](bool ring) {
+    return sizeof(float) * ((size_t)2 * K::J + (VJP ? 2 * 32 * 8 : 64 + 2 * 32 * 2 + 64 + 64) + 4 +
+                            (VJP ? 2 : 1) * (size_t)sh.n +
+                            (ring ? (size_t)K::NS * K::kStageFloats + K::kRingCtlWords : 0));
+  };
+  bool ring = VJP && l16_vjp_ring() && smem_for(true) <= kMaxDynSmem;
+  size_t smem = smem_for(ring);
   if (smem > kMaxDynSmem) return BCJR_ERR_UNSUPPORTED;
+  void (*kern)(K::Params) = pick(false, ring);
   int grid = 0;
   int rc = grid_for(kern, K::NT, smem, sh.n_seq, &grid);
   if (rc != BCJR_OK) return rc;
@@ -340,7 +359,9 @@ int run_l16(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   const size_t full_cta = sizeof(float) * (size_t)sh.n * K::J * (VJP ? 2 : 1);
   const int ck = l16_checkpoint_len(sh.n, grid, full_cta);
   if (ck) {
-    kern = pick(true);
+    ring = false;
+    smem = smem_for(false);
+    kern = pick(true, false);
     if ((rc = grid_for(kern, K::NT, smem, sh.n_seq, &grid)) != BCJR_OK) return rc;
   }
   const size_t nseg = ck ? (size_t)((sh.n + ck - 1) / ck) : 0;
@@ -352,6 +373,7 @@ int run_l16(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   K::Params P{};
   auto layout = [&](Arena& ar) {
     P.cs_tm = ar.take<float>(K::S);
+    P.cs_rg = ring ? ar.take<float>(K::S) : nullptr;
     P.hist_l = ar.take<float>((size_t)grid * hist_cta_floats);
     P.hist_a = (VJP && !ck) ? ar.take<float>((size_t)grid * hist_cta_floats) : nullptr;
     P.hist_c = ar.take<double>((size_t)grid * sh.n);
@@ -371,7 +393,9 @@ int run_l16(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   P.n_seq = sh.n_seq; P.len = sh.len; P.n = sh.n; P.ck = ck;
   P.sk = (float)std::sqrt(1.4426950408889634 / (double)a.T);
   P.two_over_T = (float)(2.0 / (double)a.T);
+  P.ring_nofill = (ring && l16_ring_test_nofill()) ? 1 : 0;
   K::make_block_codebook<<<K::S / 256, 256, 0, st>>>(a.c, P.sk, const_cast<float*>(P.cs_tm));
+  if (ring) K::make_ring_codebook<<<K::S / 256, 256, 0, st>>>(P.cs_tm, const_cast<float*>(P.cs_rg));
   kern<<<grid, K::NT, smem, st>>>(P);
   if (VJP) K::reduce_block_gc<<<K::S / 256, 256, 0, st>>>(P.gc_part, grid, a.grad_c);
   cudaError_t le = cudaGetLastError();

@@ -42,7 +42,7 @@ constexpr int kMaxWarps = kMaxThreads / 32;
 // First device-side error recorded by a kernel of this library (a status code
 // of the C interface, 0 = none); read and cleared by bcjr_get_device_error.
 __device__ int g_device_error = 0;
-constexpr int kErrTimeout = 4;   // reserved: no kernel of this version waits on a flag
+constexpr int kErrTimeout = 4;   // a bounded wait ran out (the L=16 VJP's codeword ring)
 constexpr int kErrNumeric = 5;   // a per-step posterior mass left 1 +- 1e-2, or was not finite
 __device__ __forceinline__ void record_device_error(int code) { atomicCAS(&g_device_error, 0, code); }
 // The posterior of every step sums to 1 (both sweeps are exact rewritings of

@@ -25,7 +25,8 @@
 //   Tensor memory (512 columns x 128 lanes = 65536 fp32, one per state) holds,
 //   for SOFT, the thread's codewords (read back every step without touching
 //   L2) and, for VJP, the current sequence's per-state codebook gradient
-//   (the VJP streams the codebook from L2 instead); warp w uses lanes
+//   (the VJP's backward then reads the codebook through a shared-memory ring
+//   that bulk copies fill, or streams it from L2); warp w uses lanes
 //   32 (w mod 4) .. + 31 and columns 128 (w div 4) + 16 k for block k.
 #pragma once
 #include "bcjr_kernels.cuh"
@@ -41,6 +42,7 @@ static_assert(NT / 32 == 16, "the per-step reductions combine 16 warps");
 struct Params {
   const float* w;        // [n_seq][len]
   const float* cs_tm;    // block-major scaled codebook [4096][16]
+  const float* cs_rg;    // the same in ring order (make_ring_codebook), VJP with the codeword ring
   const float* gsoft;    // [n_seq][len] (VJP)
   const float* gZ;       // [n_seq] or null (VJP)
   float* out_soft;       // [n_seq][len] or null
@@ -57,6 +59,7 @@ struct Params {
   int64_t n_seq, len;
   int n;
   float sk, two_over_T;
+  int ring_nofill;       // test hook: the ring is never filled, so its bounded waits run out
 };
 
 // ------------------------------------------------------------ tensor memory
@@ -149,6 +152,72 @@ __global__ void make_block_codebook(const float* __restrict__ c, float sk, float
   if (x >= S) return;
   const int mid = x >> 4, r = x & 15, h = ((r >> 3) << 1) | (r & 1), lo = (r >> 1) & 3;
   cs_tm[x] = sk * c[(h << 14) | (mid << 2) | lo];
+}
+
+// ------------------------------------------------------------ codeword ring
+// The VJP backward keeps the sequence's codebook gradient in tensor memory, so
+// its codewords come from global memory: through a ring of NS shared-memory
+// stages, each holding one block k of every thread (32 KB), filled by bulk
+// copies (cp.async.bulk, completion counted on the stage's mbarrier).  Every
+// warp, after its last read of a stage, adds one to the stage's release counter;
+// the sixteenth warp refills the stage with block k + NS.  A warp therefore
+// never waits for a producer, only for the copy, which was issued one block
+// earlier.  cs_rg orders each block's chunk quad-major,
+// cs_rg[((k * 4 + i) * NT + tau) * 4 + e] = cs_tm[(tau + NT k) * 16 + 4 i + e],
+// so that a warp's 16-byte shared-memory reads of one quad are consecutive.
+__global__ void make_ring_codebook(const float* __restrict__ cs_tm, float* __restrict__ cs_rg) {
+  int x = blockIdx.x * blockDim.x + threadIdx.x;
+  if (x >= S) return;
+  const int e = x & 3, tau = (x >> 2) & (NT - 1), i = (x >> 11) & 3, k = x >> 13;
+  cs_rg[x] = cs_tm[(size_t)(tau + NT * k) * 16 + 4 * i + e];
+}
+
+constexpr int NS = 2;                                   // ring stages
+constexpr int kStageFloats = 4 * NT * 4;                // one block of every thread, 32 KB
+constexpr uint32_t kStageBytes = kStageFloats * sizeof(float);
+constexpr int kRingCtlWords = 24;                       // 4 mbarriers, 4 + 4 counters, failure flag, padding
+constexpr uint64_t kRingWaitNs = 1000000000ull;        // a wait gives up after 1 s
+
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(b)), "r"(count) : "memory");
+}
+// Bulk copy of one stage; the mbarrier's phase completes when its bytes have landed.
+__device__ __forceinline__ void ring_fill(float* stage, const float* src, uint64_t* full) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(full)), "r"(kStageBytes)
+               : "memory");
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_addr(stage)),
+               "l"(src), "r"(kStageBytes), "r"(smem_addr(full))
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Waits for the phase of parity `parity` to complete; false after kRingWaitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
+  const uint32_t a = smem_addr(b);
+  if (mbar_try(a, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (!mbar_try(a, parity)) {
+    if (global_ns() - t0 > kRingWaitNs) return false;
+  }
+  return true;
+}
+__device__ __forceinline__ uint32_t ring_release(uint32_t* cnt) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;" : "=r"(old) : "r"(smem_addr(cnt)) : "memory");
+  return old;
 }
 
 // grad_c[q] = sum over CTAs of gc_part[cta][block-major index of q]
@@ -664,20 +733,29 @@ __global__ void __launch_bounds__(NT, 1) soft_kernel(Params P) {
 // exchanges the negated log rho and Bc = W / P instead.  Both renormalise the
 // posterior mass of every step (its sum drifts from 1 by the rounding of the
 // two sweeps).
-template <bool POST, bool CKPT>
+// RING: the backward's codewords through the shared-memory ring (full
+// histories only), else streamed from L2 and prefetched two units ahead.
+template <bool POST, bool CKPT, bool RING>
 __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
+  static_assert(!(RING && CKPT), "the codeword ring runs with full histories");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n = P.n;
 
   extern __shared__ __align__(16) float smem[];
-  float* sb = smem;                                    // [2][J] forward values / P or negated log rho
+  float* ring = smem;                                  // RING: [NS][kStageFloats]
+  float* sb = smem + (RING ? NS * kStageFloats : 0);   // [2][J] forward values / P or negated log rho
   float* lb[2] = {sb, sb + J};
   // per-warp partials of a step, [2 parities][32][8]:
   //   0: sum P(i) (A + Bc)   1: sum P(i) Bc   2: sum P(i)   3: min stored value
   //   4: sum G c             5: sum G
   float* rec = sb + 2 * J;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(rec + 2 * 32 * 8);  // [4]
-  float* wsc = reinterpret_cast<float*>(tslot + 4);    // n: -w'
+  // RING control: stage mbarriers, release counters, fills issued per stage, failure flag
+  uint64_t* fullb = reinterpret_cast<uint64_t*>(tslot + 4);
+  uint32_t* rcnt = reinterpret_cast<uint32_t*>(fullb + 4);
+  uint32_t* rfill = rcnt + 4;
+  uint32_t* rfail = rfill + 4;
+  float* wsc = reinterpret_cast<float*>(tslot + 4 + (RING ? kRingCtlWords : 0));   // n: -w'
   float* gsc = wsc + n;                                // n: g / sk
 
   // Per-CTA histories (see History), full or checkpointed.  Full: the forward
@@ -716,11 +794,28 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
   const float2 neg1 = f2s(-1.f);
 
   if (warp == 0) tmem_alloc512(tslot);
+  if (RING && tid == 0) {
+    for (int s2 = 0; s2 < NS; ++s2) {
+      mbar_init(&fullb[s2], 1);
+      rcnt[s2] = 0;
+      rfill[s2] = 0;
+    }
+    *rfail = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
   tmem_fence_before();
   __syncthreads();
   tmem_fence_after();
   const uint32_t tbase = tslot[0] + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(128 * (warp >> 2));
   for (int x = tid; x < S; x += NT) gcp[x] = 0.0;
+  // ring position of the next block the backward reads (the same on every thread)
+  uint32_t rstage = 0, rphase = 0;
+  bool ring_ok = true;
+  auto issue_fill = [&](uint32_t st, int k) {   // stage st <- block k
+    if (P.ring_nofill) return;
+    ring_fill(ring + st * kStageFloats, P.cs_rg + (size_t)k * kStageFloats, &fullb[st]);
+    atomicAdd(&rfill[st], 1u);
+  };
 
   // One forward step: step t-1's forward values (shared memory) and A (global
   // ping-pong) in, step t's out; history slots that are non-null receive step
@@ -886,8 +981,19 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
     // relative to rB, the posterior mean of the previous step's stored values.
     float Kt = Hbar, rB = 0.f;
     float cbn[8], cbm[8];
-    ld_cb8(cs_tm, tid, 0, cbn);
-    ld_cb8(cs_tm, tid, 1, cbm);
+    if constexpr (RING) {
+      // blocks 0 .. NS-1 of step n-1; every stage was released in the previous sequence
+      if (tid == 0) {
+        uint32_t st = rstage;
+        for (int i = 0; i < NS; ++i) {
+          issue_fill(st, i);
+          st = (st + 1 == NS) ? 0 : st + 1;
+        }
+      }
+    } else {
+      ld_cb8(cs_tm, tid, 0, cbn);
+      ld_cb8(cs_tm, tid, 1, cbm);
+    }
     // block-major input slot of step tt (tt >= 1), full or in the segment
     auto in_slot = [&](const float* full, const float* seg, int tt) -> const float* {
       if constexpr (!CKPT) return full + (size_t)(tt - 1) * J;
@@ -993,6 +1099,14 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
 #pragma unroll
       for (int k = 0; k < KB; ++k) {
         const int mid = tid + NT * k;
+        if constexpr (RING) {
+          if (ring_ok && !mbar_wait(&fullb[rstage], rphase)) {
+            record_device_error(kErrTimeout);
+            *rfail = 1;
+            ring_ok = false;
+          }
+        }
+        const float4* st4 = reinterpret_cast<const float4*>(ring + rstage * kStageFloats);
         float nr[4], bc[4];   // P and W (POST) or negated log rho and Bc
         if (last && !POST) {
           nr[0] = nr[1] = nr[2] = nr[3] = 0.f;
@@ -1028,9 +1142,13 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
 #pragma unroll
         for (int g = 0; g < 2; ++g) {          // groups h = 2g, 2g+1 side by side
           float cb[8];
+          if constexpr (RING) {
+            const float4 q0 = st4[(2 * g) * NT + tid], q1 = st4[(2 * g + 1) * NT + tid];
+            cb[0] = q0.x; cb[1] = q0.y; cb[2] = q0.z; cb[3] = q0.w;
+            cb[4] = q1.x; cb[5] = q1.y; cb[6] = q1.z; cb[7] = q1.w;
+          } else {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) { cb[i] = cbn[i]; cbn[i] = cbm[i]; }
-          {
+            for (int i = 0; i < 8; ++i) { cb[i] = cbn[i]; cbn[i] = cbm[i]; }
             // codewords two units after (k, g): block k+1 (or 0), same g
             const int nk = (k + 1 < KB) ? k + 1 : 0;
             ld_cb8(cs_tm, tid + NT * nk, g, cbm);
@@ -1107,6 +1225,22 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
           }
           tmem_st8(tbase + 16 * k + 8 * g, gcb);
         }
+        if constexpr (RING) {
+          // this warp has read block k's stage; the last of the 16 warps refills it
+          // with block k + NS (in this step or the next; none after the last step)
+          __syncwarp();
+          if (lane == 0) {
+            const uint32_t old = ring_release(&rcnt[rstage]);
+            if ((old & 15) == 15 && !(t == 0 && k + NS >= KB) && ring_ok) {
+              asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+              issue_fill(rstage, (k + NS) % KB);
+            }
+          }
+          if (++rstage == NS) {
+            rstage = 0;
+            rphase ^= 1;
+          }
+        }
         if (t >= 1) {
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
@@ -1171,6 +1305,11 @@ __global__ void __launch_bounds__(NT, 1) vjp_kernel(Params P) {
   tmem_fence_before();
   __syncthreads();
   tmem_fence_after();
+  if (RING && tid == 0 && *rfail) {
+    // after a wait that ran out: the copies still in flight land before the CTA exits
+    for (int s2 = 0; s2 < NS; ++s2)
+      if (rfill[s2] > 0) mbar_wait(&fullb[s2], (rfill[s2] - 1) & 1);
+  }
   if (warp == 0) tmem_dealloc512(tslot[0]);
 }
 

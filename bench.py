@@ -107,7 +107,7 @@ def measured_peaks():
 def kernel_variants() -> dict:
     """The library's kernel selectors as this process sees them (defaults spelled out)."""
     return {"l16_backward": os.environ.get("BCJR_L16_BWD", "post (soft), log (VJP)"),
-            "l16_vjp": os.environ.get("BCJR_L16_VJP", "one CTA per sequence"),
+            "l16_vjp": os.environ.get("BCJR_L16_VJP", "one CTA per sequence, codewords through a shared-memory ring"),
             "l16_ex2": os.environ.get("BCJR_L16_EX2", "mufu"),
             "l16_histories": os.environ.get("BCJR_L16_CKPT", "full, or sqrt(n) checkpoints beyond the scratch budget")}
 

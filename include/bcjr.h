@@ -69,7 +69,7 @@ typedef enum {
   BCJR_ERR_INVALID_ARG = 1,
   BCJR_ERR_UNSUPPORTED = 2,
   BCJR_ERR_CUDA = 3,
-  BCJR_ERR_TIMEOUT = 4,  /* reserved: no kernel of this version waits on a flag */
+  BCJR_ERR_TIMEOUT = 4,  /* recorded on the device: a bounded wait ran out */
   BCJR_ERR_NUMERIC = 5   /* recorded on the device: a step's posterior mass was off */
 } bcjr_status;
 
@@ -199,8 +199,11 @@ BCJR_API int bcjr_qat_step(float* w, const float* w_target, int64_t n_seq, int64
  * Synchronises `stream` and returns BCJR_OK, or BCJR_ERR_CUDA if the stream
  * holds a CUDA error, or the first device-side error recorded by a kernel of
  * this library since the last call (BCJR_ERR_NUMERIC: a step's posterior mass
- * left 1 +- 1e-2 or was not finite).  The flag is one per device and process,
- * shared by all streams; reading it clears it.
+ * left 1 +- 1e-2 or was not finite; BCJR_ERR_TIMEOUT: a wait of the L=16 V=1
+ * VJP for a bulk copy into its shared-memory codeword ring did not end within
+ * 1 s, after which that CTA computes on without the ring and its sequences'
+ * outputs are not usable).  The flag is one per device and process, shared by
+ * all streams; reading it clears it.
  */
 BCJR_API int bcjr_get_device_error(void* stream);
 

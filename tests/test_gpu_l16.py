@@ -1,8 +1,10 @@
 """The specialised L=16 kernels and their measured alternatives: the two-CTA
-cluster VJP against the single-CTA VJP, the posterior-space backward sweeps
-against the log-domain ones, both against the oracle; and run-to-run bit
-reproducibility of every L=16 kernel (soft codeword, VJP, posterior argmax and
-Viterbi; V=1 and V=2).
+cluster VJP against the single-CTA VJP, the VJP backward's codeword ring
+against codewords streamed from L2, the posterior-space backward sweeps against
+the log-domain ones, all against the oracle; run-to-run bit reproducibility of
+every L=16 kernel (soft codeword, VJP, posterior argmax and Viterbi; V=1 and
+V=2); and the ring's bounded wait, made to run out by a test hook, reporting
+BCJR_ERR_TIMEOUT with the context still usable.
 
 All calls go through libbcjr.so (include/bcjr.h) via the ctypes binding.
 """
@@ -42,7 +44,7 @@ def test_l16_cluster_vjp_matches_single_cta_vjp(monkeypatch):
     assert_grad(gc_sub.cpu().numpy(), rv["grad_c"], "grad_c")
 
 
-@pytest.mark.parametrize("variant", [{}, {"BCJR_L16_VJP": "cluster"}, {"BCJR_L16_BWD": "post"}])
+@pytest.mark.parametrize("variant", [{}, {"BCJR_L16_VJP": "cluster"}, {"BCJR_L16_VJP": "l2"}, {"BCJR_L16_BWD": "post"}])
 def test_l16_vjp_single_sequence_and_short(monkeypatch, variant):
     """One sequence (one CTA or cluster busy, the rest idle) and n = 1 and 2 steps."""
     for key, val in variant.items():
@@ -65,7 +67,7 @@ def _twice(fn):
     return a, b
 
 
-@pytest.mark.parametrize("variant", [{}, {"BCJR_L16_VJP": "cluster"}, {"BCJR_L16_BWD": "post"},
+@pytest.mark.parametrize("variant", [{}, {"BCJR_L16_VJP": "cluster"}, {"BCJR_L16_VJP": "l2"}, {"BCJR_L16_BWD": "post"},
                                      {"BCJR_L16_BWD": "log"}, {"BCJR_L16_EX2": "fma"}])
 def test_l16_v1_runs_are_bit_identical(monkeypatch, variant):
     """L=16, k=2, V=1: soft codeword, logZ, argmax and VJP of 200 sequences
@@ -147,7 +149,7 @@ def longest_low_t_case():
     return w, c, g, ref, rv
 
 
-@pytest.mark.parametrize("variant", [{}, {"BCJR_L16_BWD": "post"}, {"BCJR_L16_BWD": "log"},
+@pytest.mark.parametrize("variant", [{}, {"BCJR_L16_BWD": "post"}, {"BCJR_L16_BWD": "log"}, {"BCJR_L16_VJP": "l2"},
                                      {"BCJR_L16_EX2": "fma"}, {"BCJR_GENERIC_ONLY": "1"}])
 def test_l16_variants_longest_sequences_low_temperature(monkeypatch, variant, longest_low_t_case):
     """len = 8192 at T = 0.01 with a biased upstream gradient, where the log
@@ -192,3 +194,45 @@ def test_l16_checkpointed_histories_are_bit_identical(monkeypatch, variant, n, K
     ck = run()
     for a, b in zip(full, ck):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("bwd", ["log", "post"])
+def test_l16_codeword_ring_equals_l2_stream(monkeypatch, bwd):
+    """The VJP backward's codewords through the shared-memory ring (default) and
+    streamed from L2 (BCJR_L16_VJP=l2) are the same numbers fed to the same
+    arithmetic: bit-identical dl/dw and dl/dc on 300 sequences of 37 steps (the
+    ring's stages wrap within and across sequences: 8 x 37 blocks per
+    sequence), with a logZ gradient, and both against the oracle on some rows."""
+    monkeypatch.setenv("BCJR_L16_BWD", bwd)
+    w, c, g = I.random_case(16, 2, 1, 300, 37, seed=1500)
+    gZ = torch.randn(300, generator=torch.Generator().manual_seed(15))
+    wd, cd, gd, gzd = w.to(DEV), c.to(DEV), g.to(DEV), gZ.to(DEV)
+    ring = [x.clone() for x in lib.vjp(wd, cd, 16, 2, 1, 0.1, gd, gzd)]
+    assert lib.get_device_error() == 0
+    monkeypatch.setenv("BCJR_L16_VJP", "l2")
+    l2 = [x.clone() for x in lib.vjp(wd, cd, 16, 2, 1, 0.1, gd, gzd)]
+    assert lib.get_device_error() == 0
+    for a, b in zip(ring, l2):
+        assert torch.equal(a, b)
+    rows = [0, 147, 148, 299]
+    rv = oracle.vjp(w[rows], c, 16, 2, 1, 0.1, g[rows], gZ[rows])
+    assert_grad(ring[0].cpu().numpy()[rows], rv["grad_w"], "grad_w")
+
+
+def test_l16_ring_wait_runs_out_and_reports_timeout(monkeypatch):
+    """With the test hook BCJR_L16_RING_TEST_NOFILL=1 no bulk copy is issued, so
+    every CTA's first wait for a ring stage runs out after its 1 s bound: the call
+    returns, bcjr_get_device_error reports BCJR_ERR_TIMEOUT, and the next call
+    on the same context is correct (against the oracle) with the flag clear."""
+    w, c, g = I.random_case(16, 2, 1, 3, 6, seed=1501)
+    wd, cd, gd = w.to(DEV), c.to(DEV), g.to(DEV)
+    monkeypatch.setenv("BCJR_L16_RING_TEST_NOFILL", "1")
+    lib.vjp(wd, cd, 16, 2, 1, 0.2, gd)
+    assert lib.get_device_error() == lib.BCJR_ERR_TIMEOUT
+    assert lib.get_device_error() == 0
+    monkeypatch.delenv("BCJR_L16_RING_TEST_NOFILL")
+    gw, gc = lib.vjp(wd, cd, 16, 2, 1, 0.2, gd)
+    assert lib.get_device_error() == 0
+    rv = oracle.vjp(w, c, 16, 2, 1, 0.2, g)
+    assert_grad(gw.cpu().numpy(), rv["grad_w"], "grad_w")
+    assert_grad(gc.cpu().numpy(), rv["grad_c"], "grad_c")
