@@ -76,7 +76,7 @@ VITERBI_LEDGERS = {(2, 1): {"fp32": 3.0, "alu": 0.75}, (2, 2): {"fp32": 6.0, "al
 # history traffic as a full launch); set to None whenever the kernel changes.
 # (A 16-sequence capture of the V=2 kernels keeps their histories in L2, so it
 # does not scale to a full launch; their traffic is reported as null.)
-TRAFFIC_PER_SEQ = {"vjp": (452.24e6 + 548.47e6) / 16, "soft": (173.51e6 + 271.59e6) / 16}
+TRAFFIC_PER_SEQ = {"vjp": (457.83e6 + 548.85e6) / 16, "soft": (179.55e6 + 271.94e6) / 16}
 FP32_PER_CLK_SM = 128.0   # FFMA lanes per SM per clock (measured by microbenchmark: 123.5 FFMA, 126 FFMA2)
 MUFU_PER_CLK_SM = 16.0    # ex2 per SM per clock (measured by microbenchmark: 15.99)
 ALU_PER_CLK_SM = 64.0     # compare / min-max lanes per SM per clock (nominal)
