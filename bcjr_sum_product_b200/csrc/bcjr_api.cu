@@ -5,6 +5,7 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include <cuda_runtime.h>
@@ -34,6 +35,10 @@ bool fault_alloc() {
   const char* e = std::getenv("BCJR_FAULT_ALLOC");
   return e && e[0] == '1';
 }
+
+// Kernels this library has launched in the process (bcjr_launch_count).
+std::atomic<uint64_t> g_launch_count{0};
+void counted_launch(int n = 1) { g_launch_count.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
 // Library-private stream-ordered pool per device.  Scratch freed at the end of
 // a call stays mapped in the pool (release threshold = unlimited), so the next
@@ -308,8 +313,12 @@ int run_l16c_vjp(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   P.two_over_T = (float)(2.0 / (double)a.T);
   cfg.gridDim = dim3((unsigned)(K::NC * ncl), 1, 1);
   bcjr::l16::make_block_codebook<<<K::S / 256, 256, 0, st>>>(a.c, P.sk, const_cast<float*>(P.cs_tm));
+  counted_launch();
   cudaError_t ke = cudaLaunchKernelEx(&cfg, K::vjp_kernel, P);
-  if (ke == cudaSuccess) bcjr::l16::reduce_block_gc<<<K::S / 256, 256, 0, st>>>(P.gc_part, ncl, a.grad_c);
+  if (ke == cudaSuccess) {
+    bcjr::l16::reduce_block_gc<<<K::S / 256, 256, 0, st>>>(P.gc_part, ncl, a.grad_c);
+    counted_launch(2);
+  }
   cudaError_t le = cudaGetLastError();
   cudaError_t fe = cudaFreeAsync(mem, st);
   if (ke != cudaSuccess || le != cudaSuccess || fe != cudaSuccess) return BCJR_ERR_CUDA;
@@ -398,6 +407,7 @@ int run_l16(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   if (ring) K::make_ring_codebook<<<K::S / 256, 256, 0, st>>>(P.cs_tm, const_cast<float*>(P.cs_rg));
   kern<<<grid, K::NT, smem, st>>>(P);
   if (VJP) K::reduce_block_gc<<<K::S / 256, 256, 0, st>>>(P.gc_part, grid, a.grad_c);
+  counted_launch(2 + (ring ? 1 : 0) + (VJP ? 1 : 0));
   cudaError_t le = cudaGetLastError();
   cudaError_t fe = cudaFreeAsync(mem, st);
   if (le != cudaSuccess || fe != cudaSuccess) return BCJR_ERR_CUDA;
@@ -452,6 +462,7 @@ int run_l16v2(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
                                                   const_cast<float2*>(P.cf1), const_cast<float2*>(P.cb1));
   kern<<<grid, K::NT, smem, st>>>(P);
   if (VJP) K::reduce_gc<<<2 * K::S / 256, 256, 0, st>>>(P.gc_part, grid, a.grad_c);
+  counted_launch(VJP ? 3 : 2);
   cudaError_t le = cudaGetLastError();
   cudaError_t fe = cudaFreeAsync(mem, st);
   if (le != cudaSuccess || fe != cudaSuccess) return BCJR_ERR_CUDA;
@@ -508,6 +519,7 @@ int run_sweep(const Shape& sh, const SweepArgs& a, cudaStream_t st) {
   bcjr::scale_codebook_kernel<<<(sv + 255) / 256, 256, 0, st>>>(a.c, sv, P.sk, const_cast<float*>(P.cs));
   kern<<<grid, threads, smem, st>>>(P);
   if (VJP) bcjr::reduce_gc_kernel<<<(sv + 255) / 256, 256, 0, st>>>(P.gc_part, grid, sv, a.grad_c);
+  counted_launch(VJP ? 3 : 2);
   cudaError_t le = cudaGetLastError();
   cudaError_t fe = cudaFreeAsync(mem, st);
   if (le != cudaSuccess || fe != cudaSuccess) return BCJR_ERR_CUDA;
@@ -557,6 +569,7 @@ int run_viterbi_l16(const Shape& sh, const float* w, const float* c, int32_t* ou
   P.n_seq = sh.n_seq; P.len = sh.len; P.n = sh.n; P.tb = (int)tb;
   K::make_block_codebook<<<K::S / 256, 256, 0, st>>>(c, 1.0f, const_cast<float*>(P.cb_raw));
   K::viterbi_kernel<<<grid, K::NT, smem, st>>>(P);
+  counted_launch(2);
   cudaError_t le = cudaGetLastError();
   cudaError_t fe = cudaFreeAsync(mem, st);
   if (le != cudaSuccess || fe != cudaSuccess) return BCJR_ERR_CUDA;
@@ -600,6 +613,7 @@ int run_viterbi_l16v2(const Shape& sh, const float* w, const float* c, int32_t* 
   P.n_seq = sh.n_seq; P.len = sh.len; P.n = sh.n; P.tb = (int)tb;
   K::make_codebooks<<<K::CB4 / 256, 256, 0, st>>>(c, 1.0f, cf, cbk, cf1, cb1);   // raw codewords
   K::viterbi_kernel<<<grid, K::NT, smem, st>>>(P);
+  counted_launch(2);
   cudaError_t le = cudaGetLastError();
   cudaError_t fe = cudaFreeAsync(mem, st);
   if (le != cudaSuccess || fe != cudaSuccess) return BCJR_ERR_CUDA;
@@ -638,6 +652,7 @@ int run_viterbi(const Shape& sh, const float* w, const float* c, int32_t* out_st
   P.n_seq = sh.n_seq; P.len = sh.len; P.L = sh.L; P.n = sh.n; P.J = sh.J; P.S = sh.S;
   P.state_in_smem = in_smem ? 1 : 0;
   kern<<<grid, threads, smem, st>>>(P);
+  counted_launch();
   cudaError_t le = cudaGetLastError();
   cudaError_t fe = cudaFreeAsync(mem, st);
   if (le != cudaSuccess || fe != cudaSuccess) return BCJR_ERR_CUDA;
@@ -738,6 +753,7 @@ int bcjr_qat_step(float* w, const float* w_target, int64_t n_seq, int64_t len, i
   if ((rc = scratch_alloc(&g, sizeof(float) * (size_t)nw, st))) return rc;
   bcjr::recon_grad_kernel<<<(unsigned)std::min<int64_t>(n_seq, 148 * 64), 256, 0, st>>>(
       out_soft, w_target, n_seq, len, static_cast<float*>(g), out_loss);
+  counted_launch();
   SweepArgs b{w, codebook, T, static_cast<float*>(g), nullptr, nullptr, nullptr, nullptr, grad_w, grad_codebook};
   rc = run_sweep<bcjr::MODE_VJP>(sh, b, st);
   if (rc == BCJR_OK) {
@@ -745,11 +761,14 @@ int bcjr_qat_step(float* w, const float* w_target, int64_t n_seq, int64_t len, i
     bcjr::sgd_kernel<<<(unsigned)std::min<int64_t>((nw + 255) / 256, 148 * 16), 256, 0, st>>>(w, grad_w, lr_w, nw);
     if (lr_c != 0.f)
       bcjr::sgd_kernel<<<(unsigned)((sv + 255) / 256), 256, 0, st>>>(codebook, grad_codebook, lr_c, sv);
+    counted_launch(lr_c != 0.f ? 2 : 1);
     if (cudaGetLastError() != cudaSuccess) rc = BCJR_ERR_CUDA;
   }
   if (cudaFreeAsync(g, st) != cudaSuccess && rc == BCJR_OK) rc = BCJR_ERR_CUDA;
   return rc;
 }
+
+uint64_t bcjr_launch_count(void) { return g_launch_count.load(std::memory_order_relaxed); }
 
 int bcjr_get_device_error(void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -884,6 +903,7 @@ extern "C" int bcjr_soft_codeword_noalloc(const float* w, int64_t n_seq, int64_t
   const int sv = (int)SV;
   bcjr::scale_codebook_kernel<<<(sv + 255) / 256, 256, 0, st>>>(codebook, sv, P.sk, const_cast<float*>(P.cs));
   kern<<<grid, threads, smem, st>>>(P);
+  counted_launch(2);
   return cudaGetLastError() == cudaSuccess ? BCJR_OK : BCJR_ERR_CUDA;
 }
 

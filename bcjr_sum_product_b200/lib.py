@@ -24,7 +24,7 @@ BCJR_ERR_TIMEOUT = 4
 BCJR_ERR_NUMERIC = 5
 
 EXPORTS = ("bcjr_soft_codeword", "bcjr_vjp", "viterbi_decode", "bcjr_posterior_argmax",
-           "bcjr_get_device_error", "bcjr_strerror", "bcjr_version")
+           "bcjr_get_device_error", "bcjr_launch_count", "bcjr_strerror", "bcjr_version")
 
 
 class BcjrError(RuntimeError):
@@ -59,6 +59,8 @@ def load(path: str = LIB_PATH):
             lib.bcjr_strerror.restype = ctypes.c_char_p
             lib.bcjr_version.argtypes = []
             lib.bcjr_version.restype = ctypes.c_char_p
+            lib.bcjr_launch_count.argtypes = []
+            lib.bcjr_launch_count.restype = ctypes.c_uint64
             for name in ("bcjr_soft_codeword", "bcjr_vjp", "viterbi_decode", "bcjr_posterior_argmax",
                          "bcjr_qat_step", "bcjr_get_device_error"):
                 getattr(lib, name).restype = ctypes.c_int
@@ -68,6 +70,11 @@ def load(path: str = LIB_PATH):
 
 def strerror(status: int) -> str:
     return load().bcjr_strerror(int(status)).decode()
+
+
+def launch_count() -> int:
+    """bcjr_launch_count: kernels the library has launched in this process."""
+    return int(load().bcjr_launch_count())
 
 
 def version() -> str:

@@ -207,6 +207,11 @@ BCJR_API int bcjr_qat_step(float* w, const float* w_target, int64_t n_seq, int64
  */
 BCJR_API int bcjr_get_device_error(void* stream);
 
+/* Number of kernels this library has launched in this process, on all devices
+ * and streams (launches issued, counted on the host; a call that fails before
+ * launching adds nothing).  For accounting, e.g. the launches of a timed region. */
+BCJR_API uint64_t bcjr_launch_count(void);
+
 /* Static string for a status code. */
 BCJR_API const char* bcjr_strerror(int status);
 

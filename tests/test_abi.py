@@ -23,7 +23,7 @@ def _declared_functions():
 def test_header_declares_the_boundary():
     names = _declared_functions()
     for n in ("bcjr_soft_codeword", "bcjr_vjp", "viterbi_decode", "bcjr_posterior_argmax",
-              "bcjr_get_device_error", "bcjr_strerror", "bcjr_version"):
+              "bcjr_get_device_error", "bcjr_launch_count", "bcjr_strerror", "bcjr_version"):
         assert n in names
 
 
@@ -83,3 +83,14 @@ def test_binding_rejects_host_tensors():
     from bcjr_sum_product_b200 import lib
     with pytest.raises(TypeError):
         lib.soft_codeword(torch.zeros(2, 8), torch.zeros(256), 8, 2, 1, 0.5)
+
+
+def test_rejected_calls_launch_nothing():
+    """bcjr_launch_count counts kernels issued: calls that fail argument or
+    shape validation (no GPU needed) leave it unchanged."""
+    from bcjr_sum_product_b200 import lib
+    n0 = lib.launch_count()
+    assert n0 >= 0
+    assert _call_soft(L=17) == lib.BCJR_ERR_UNSUPPORTED
+    assert _call_soft(length=0) == lib.BCJR_ERR_INVALID_ARG
+    assert lib.launch_count() == n0

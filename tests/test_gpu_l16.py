@@ -236,3 +236,21 @@ def test_l16_ring_wait_runs_out_and_reports_timeout(monkeypatch):
     rv = oracle.vjp(w, c, 16, 2, 1, 0.2, g)
     assert_grad(gw.cpu().numpy(), rv["grad_w"], "grad_w")
     assert_grad(gc.cpu().numpy(), rv["grad_c"], "grad_c")
+
+
+def test_launch_count_per_call(monkeypatch):
+    """bcjr_launch_count over single calls at L=16, k=2, V=1: the soft codeword
+    is the block-codebook staging plus the sweep (2); the VJP adds the ring's
+    codebook copy and the gradient reduction (4), or 3 with BCJR_L16_VJP=l2."""
+    w, c, g = I.random_case(16, 2, 1, 4, 16, seed=1502)
+    wd, cd, gd = w.to(DEV), c.to(DEV), g.to(DEV)
+    n0 = lib.launch_count()
+    lib.soft_codeword(wd, cd, 16, 2, 1, 0.5)
+    n1 = lib.launch_count()
+    lib.vjp(wd, cd, 16, 2, 1, 0.5, gd)
+    n2 = lib.launch_count()
+    monkeypatch.setenv("BCJR_L16_VJP", "l2")
+    lib.vjp(wd, cd, 16, 2, 1, 0.5, gd)
+    n3 = lib.launch_count()
+    assert lib.get_device_error() == 0
+    assert (n1 - n0, n2 - n1, n3 - n2) == (2, 4, 3)
